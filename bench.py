@@ -1,0 +1,447 @@
+"""Benchmark: paged decode attention KV-read GB/s on the Qwen3-4B-shaped decode
+batch (64 slots, 32/8 heads, d=128, page 16, lengths U[128,4096]), plus the
+other workloads (mixed prefill+decode tokens/s, long-context split-K,
+fragmented large batch, tiny decode).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workloads all|none|name,...]
+
+A step is one pass of the hot path over one batch: kv_append of the step's new
+K/V rows, then attention (chunked prefill for prompt chunks, decode with its
+split-K partition + combine for decode rows).  Inputs are resident in HBM
+when the timed region starts; the KV a step reads is larger than the 126 MB
+L2, so no flush is needed between steps.  Under torchrun each rank runs its
+own batch (requests shard across GPUs with no data-path collective: weak
+scaling); the step time is the max over ranks.
+
+--impl reference times the CPU oracle (the plain fp64 definition) on a
+bounded sample of the same workload, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import make_workload  # noqa: E402
+
+HBM_NOMINAL_GBS = 8000.0
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+METRIC = "paged decode attention KV-read GB/s (% of 8 TB/s HBM); mixed-batch tokens/s"
+HEADLINE = "qwen3_decode"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index):
+        self.index, self.samples, self.reasons, self.max_mhz = index, [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: record why
+            self.nv, self.err = None, str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- GPU side
+class GpuWorkload:
+    """Device buffers for one workload: pools with every request's context
+    (drawn on the GPU, seeded), and the step's inputs (host-generated)."""
+
+    def __init__(self, pkv, torch, w, seed=4321):
+        self.pkv, self.torch, self.w = pkv, torch, w
+        dev = "cuda"
+        self.k_pool = torch.full(w.pool_shape(), float("nan"), dtype=torch.bfloat16, device=dev)
+        self.v_pool = torch.full_like(self.k_pool, float("nan"))
+        gen = torch.Generator(device=dev).manual_seed(seed)
+        ids = list(range(w.B))
+        at = 0
+        while at < len(ids):
+            grp, toks = [], 0
+            while at < len(ids) and (not grp or toks < (1 << 18)):
+                grp.append(ids[at]); toks += int(w.ctx_lens[ids[at]]); at += 1
+            slots = w.ctx_slots(grp)
+            if len(slots):
+                k = torch.randn((len(slots), w.num_kv_heads, w.head_dim), generator=gen, device=dev)
+                if w.k_rms_norm:
+                    k = k / k.pow(2).mean(-1, keepdim=True).sqrt()
+                v = torch.randn((len(slots), w.num_kv_heads, w.head_dim), generator=gen, device=dev)
+                pkv.pkv_kv_append(k.bfloat16().contiguous(), v.bfloat16().contiguous(),
+                                  self.i32(slots), self.k_pool, self.v_pool)
+        # step inputs, as host arrays (pinned for the end-to-end leg) and device copies
+        k, v, s = w.batch_new()
+        dec, pre = list(w.decode_ids), list(w.prefill_ids)
+        self.host = {
+            "k_new": self.bits(k), "v_new": self.bits(v), "slots": torch.from_numpy(s),
+            "pt_dec": torch.from_numpy(np.ascontiguousarray(w.page_table[dec])),
+            "len_dec": torch.from_numpy(np.ascontiguousarray(w.kv_lens[dec])),
+        }
+        if dec:
+            self.host["q_dec"] = self.bits(w.batch_q(dec))
+        if pre:
+            self.host.update({
+                "q_pre": self.bits(w.batch_q(pre)),
+                "cu_q": torch.from_numpy(w.cu_q_lens(pre)),
+                "ctx_pre": torch.from_numpy(np.ascontiguousarray(w.ctx_lens[pre])),
+                "pt_pre": torch.from_numpy(np.ascontiguousarray(w.page_table[pre])),
+            })
+        self.host = {k: t.pin_memory() for k, t in self.host.items()}
+        self.dev = {k: t.to(dev) for k, t in self.host.items()}
+        self.dec, self.pre = dec, pre
+        self.max_q = int(w.new_lens[pre].max()) if pre else 0
+        if dec:
+            self.ws = pkv.decode_workspace(len(dec), w.num_q_heads, w.head_dim,
+                                           w.max_pages * w.page_size, 0)
+            self.out_dec = torch.empty_like(self.dev["q_dec"])
+            self.out_dec_host = torch.empty_like(self.out_dec, device="cpu").pin_memory()
+        if pre:
+            self.out_pre = torch.empty_like(self.dev["q_pre"])
+            self.out_pre_host = torch.empty_like(self.out_pre, device="cpu").pin_memory()
+        torch.cuda.synchronize()
+
+    def bits(self, a):
+        return self.torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(self.torch.bfloat16)
+
+    def i32(self, a):
+        return self.torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+    def launches_per_step(self):
+        return 1 + (2 if self.dec else 0) + (1 if self.pre else 0)
+
+    def step(self, d, ev=None):
+        """One pass of the hot path on device buffers d; ev optionally brackets
+        the prefill and decode calls with CUDA events."""
+        pkv, w = self.pkv, self.w
+        pkv.pkv_kv_append(d["k_new"], d["v_new"], d["slots"], self.k_pool, self.v_pool)
+        if self.pre:
+            if ev is not None:
+                ev["pre"][0].record()
+            pkv.pkv_paged_attn_chunked_prefill(d["q_pre"], d["cu_q"], d["ctx_pre"], self.k_pool,
+                                               self.v_pool, d["pt_pre"], w.scale, self.max_q,
+                                               out=self.out_pre)
+            if ev is not None:
+                ev["pre"][1].record()
+        if self.dec:
+            if ev is not None:
+                ev["dec"][0].record()
+            pkv.pkv_paged_attn_decode(d["q_dec"], self.k_pool, self.v_pool, d["pt_dec"],
+                                      d["len_dec"], w.scale, 0, workspace=self.ws, out=self.out_dec)
+            if ev is not None:
+                ev["dec"][1].record()
+
+    def step_e2e(self):
+        """Same step through the public API from pinned host buffers: H2D of the
+        step's inputs, the kernels, D2H of the outputs."""
+        for k, t in self.host.items():
+            self.dev[k].copy_(t, non_blocking=True)
+        self.step(self.dev)
+        if self.dec:
+            self.out_dec_host.copy_(self.out_dec, non_blocking=True)
+        if self.pre:
+            self.out_pre_host.copy_(self.out_pre, non_blocking=True)
+
+    def io_bytes(self):
+        h2d = sum(t.numel() * t.element_size() for t in self.host.values())
+        d2h = (self.out_dec.numel() * 2 if self.dec else 0) + (self.out_pre.numel() * 2 if self.pre else 0)
+        return h2d, d2h
+
+
+def prefill_flops(w):
+    """QK^T and PV multiply-adds of the causal chunks (2 flops each)."""
+    tot = 0
+    for r in w.prefill_ids:
+        c, n = int(w.ctx_lens[r]), int(w.new_lens[r])
+        keys = n * c + n * (n + 1) // 2  # row i sees c + i + 1 keys
+        tot += 4 * keys * w.num_q_heads * w.head_dim
+    return tot
+
+
+def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
+    w = make_workload(name, 0)
+    g = GpuWorkload(pkv, torch, w)
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    evs = [{"pre": (mk(), mk()), "dec": (mk(), mk())} for _ in range(steps)]
+    for _ in range(warmup):
+        g.step(g.dev)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = mk(), mk()
+    with ClockSampler(clocks_index) as clk:
+        t0.record()
+        for i in range(steps):
+            g.step(g.dev, evs[i])
+        t1.record()
+        torch.cuda.synchronize()
+    total_ms = t0.elapsed_time(t1)
+    per = {"pre": [], "dec": []}
+    for i in range(steps):
+        if g.pre:
+            per["pre"].append(evs[i]["pre"][0].elapsed_time(evs[i]["pre"][1]))
+        if g.dec:
+            per["dec"].append(evs[i]["dec"][0].elapsed_time(evs[i]["dec"][1]))
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    # end-to-end through the public API with host buffers
+    for _ in range(warmup):
+        g.step_e2e()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.step_e2e()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    flags = pkv.pkv_device_error_flags(clear=True)
+    if flags:
+        raise RuntimeError(f"device error flags {flags:#x} during {name}")
+    h2d, d2h = g.io_bytes()
+    res = {
+        "w": w, "ms_per_step": total_ms / steps, "e2e_ms_per_step": e2e_ms / steps,
+        "dec_ms": statistics.mean(per["dec"]) if per["dec"] else None,
+        "pre_ms": statistics.mean(per["pre"]) if per["pre"] else None,
+        "kv_bytes_dec": w.kv_bytes_read(w.decode_ids), "kv_bytes_pre": w.kv_bytes_read(w.prefill_ids),
+        "tokens": int(w.new_lens.sum()), "flops_pre": prefill_flops(w),
+        "launches": g.launches_per_step(), "clocks": clk.summary(), "h2d": h2d, "d2h": d2h,
+    }
+    del g
+    torch.cuda.empty_cache()
+    return res
+
+
+# --------------------------------------------------------------- CPU side
+def _oracle_one_request(oracle, w, r):
+    """Build request r's pages for the oracle (its context plus this step's
+    row, in a pool of just its pages) and return the inputs of one decode."""
+    pages = w.page_table[r][w.page_table[r] >= 0]
+    table = np.arange(len(pages), dtype=np.int32)[None, :]
+    P = w.page_size
+    kp = np.full((len(pages), w.num_kv_heads, P, w.head_dim), 0x7FC0, np.uint16)
+    vp = kp.copy()
+    L = int(w.kv_lens[r])
+    pos = np.arange(L)
+    slots = (pos // P) * P + pos % P  # pages renumbered 0.. in table order
+    kc, vc = w.ctx_rows(r)
+    kn, vn = w.new_rows(r)
+    oracle.kv_append(kp, vp, np.concatenate([kc, kn]), np.concatenate([vc, vn]), slots, P)
+    return w.q_rows(r)[None, 0], kp, vp, table, np.array([L], np.int32)
+
+
+def cpu_oracle_rate(name, budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole
+    decode requests until ~budget_s of CPU time, one thread.  Returns
+    (KV GB/s, seconds, sample description)."""
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        limit = None
+    import oracle
+    w = make_workload(name, 0)
+    dec = list(w.decode_ids)
+    order = list(np.random.default_rng(0).permutation(dec))
+    done, secs, nbytes = [], 0.0, 0
+    try:
+        while order and secs < budget_s:
+            r = int(order.pop())
+            q, kp, vp, table, lens = _oracle_one_request(oracle, w, r)
+            t = time.perf_counter()
+            oracle.decode_attention(q, kp, vp, table, lens, w.page_size, w.scale)
+            secs += time.perf_counter() - t
+            done.append(r)
+            nbytes += w.kv_bytes_read([r])
+    finally:
+        if limit is not None:
+            limit.unregister() if hasattr(limit, "unregister") else limit.__exit__(None, None, None)
+    return (nbytes / secs / 1e9, secs,
+            f"{len(done)} of {len(dec)} decode requests of {name} ({nbytes / 1e6:.1f} MB KV), 1 thread")
+
+
+def reference_arm(args):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    steps, warmup = args.steps, args.warmup
+    per_step = max(2.0, 60.0 / max(1, steps + warmup))
+    rates = []
+    for i in range(warmup + steps):
+        rate, secs, sample = cpu_oracle_rate(HEADLINE, budget_s=per_step)
+        if i >= warmup:
+            rates.append((rate, secs))
+    value = statistics.mean(r for r, _ in rates)
+    w = make_workload(HEADLINE, 0)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warmup,
+        "ms_per_step": 1000 * statistics.mean(s for _, s in rates), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": HEADLINE, **{k: v for k, v in w.describe().items() if k != "workload"}},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# -------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workloads", default="all",
+                    help="extra workloads to measure besides the headline: all, none, or a list")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    dist = None
+    rank, world = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    import paged_kv_attention_37_b200 as pkv
+
+    hbm, tf_burst, tf_sust, peak_src = peaks()
+    head = measure(pkv, torch, HEADLINE, args.steps, args.warmup, dist, local)
+    extra = {}
+    names = [] if args.workloads == "none" else (
+        [n for n in ("tiny_decode", "mixed_prefill_decode", "splitk_long", "frag_large")]
+        if args.workloads == "all" else [n for n in args.workloads.split(",") if n])
+    for n in names:
+        r = measure(pkv, torch, n, args.steps, args.warmup, dist, local)
+        e = {"ms_per_step": r["ms_per_step"], "tokens_per_step": r["tokens"],
+             "tokens_per_s": world * r["tokens"] / (r["ms_per_step"] / 1e3),
+             "e2e_ms_per_step": r["e2e_ms_per_step"]}
+        if r["dec_ms"]:
+            gbs = r["kv_bytes_dec"] / (r["dec_ms"] / 1e3) / 1e9
+            e.update({"decode_kv_bytes": r["kv_bytes_dec"], "decode_ms": r["dec_ms"],
+                      "decode_kv_gbs": gbs, "decode_pct_of_8TBs": 100 * gbs / HBM_NOMINAL_GBS,
+                      "decode_frac_of_measured_hbm": gbs / hbm})
+        if r["pre_ms"]:
+            tfs = r["flops_pre"] / (r["pre_ms"] / 1e3) / 1e12
+            e.update({"prefill_ms": r["pre_ms"], "prefill_flops": r["flops_pre"],
+                      "prefill_tflops": tfs, "prefill_frac_of_measured_bf16": tfs / tf_sust})
+        e["step_kv_gbs"] = (r["kv_bytes_dec"] + r["kv_bytes_pre"]) / (r["ms_per_step"] / 1e3) / 1e9
+        e["clocks"] = r["clocks"]
+        extra[n] = e
+
+    w = head["w"]
+    kv_bytes = head["kv_bytes_dec"]
+    value = world * kv_bytes / (head["ms_per_step"] / 1e3) / 1e9
+    achieved = kv_bytes / (head["dec_ms"] / 1e3) / 1e9
+    e2e_value = world * kv_bytes / (head["e2e_ms_per_step"] / 1e3) / 1e9
+    if rank != 0:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+    cpu_rate, cpu_secs, sample = cpu_oracle_rate(HEADLINE, args.cpu_budget) if world == 1 else (None, None, None)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32",
+        "data": "synthetic",
+        "config": {"workload": HEADLINE, **{k: v for k, v in w.describe().items() if k != "workload"},
+                   "kv_bytes_per_step": kv_bytes, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (KV read per step > 126 MB), no flush"},
+        "pct_of_8TBs": 100 * value / HBM_NOMINAL_GBS,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "kernel": "decode split-K partition + combine (one pkv_paged_attn_decode call)",
+                     "peak_source": f"{peak_src} hbm_gbs", "pct_of_8TBs": 100 * achieved / HBM_NOMINAL_GBS},
+        "cpu_baseline": ({"value": cpu_rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                          "sample": sample, "seconds": cpu_secs} if cpu_rate else None),
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": head["h2d"],
+                "d2h_bytes_per_step": head["d2h"], "ms_per_step": head["e2e_ms_per_step"]},
+        "gpu_launches": head["launches"] * args.steps,
+        "clocks": head["clocks"],
+        "workloads": extra,
+    }
+    print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,223 @@
+/*
+ * pkv.h -- C ABI of a paged KV-cache attention library for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation is attention computed directly on a paged KV cache: K and V
+ * rows live in a shared pool of fixed-size pages, each request owns a page
+ * table listing its pages in logical order, and attention reads the pages
+ * through that table, with no contiguous copy of the cache and no score
+ * matrix in memory.  Sources, by page and section:
+ *   - page pool, page tables, on-demand pages, and "paged FlashAttention"
+ *     (paging fused with an online softmax in one kernel): tiny-llm source
+ *     reading, week 3, section "Paged KV Cache"; the same course's blog
+ *     summary, week 3 ("Direct paged attention + paged FlashAttention");
+ *   - mixed prefill/decode batches and chunked prefill: tiny-llm source
+ *     reading, sections "Continuous Batching" and "Chunked Prefill";
+ *   - GQA: tiny-llm source reading, week 1;
+ *   - online softmax (FlashAttention-style) and PagedAttention in CUDA:
+ *     tiny-vllm article, section "From Safetensors to PagedAttention";
+ *   - split-K over the KV length (flash-decoding): mini-vllm advanced series
+ *     design, section 4, Phase B, adv04.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Types: bf16 tensors are raw IEEE bfloat16 (2 bytes).  int32 arrays are
+ * little-endian int32_t.
+ *
+ * Pools: k_pool and v_pool are separate arrays, each laid out
+ *   [num_pages][num_kv_heads][page_size][head_dim]  (bf16, row-major),
+ * so the rows of one (page, KV head) form one contiguous block.  A slot
+ * number names one token row of the pool: slot = page * page_size + offset.
+ *
+ * Page tables: page_table is [batch][max_pages] int32, row r listing request
+ * r's pool pages in logical order; token j of request r is row j % page_size
+ * of page page_table[r][j / page_size].  Entries past a request's last page
+ * are never read.
+ *
+ * GQA: num_q_heads must be a multiple of num_kv_heads; query head h reads KV
+ * head h / (num_q_heads / num_kv_heads).  Supported group sizes: 1, 2, 4, 8.
+ * Supported head_dim: 64, 128.  Supported page_size: 16, 32.
+ *
+ * Memory and ownership: every pointer except the host-side pool descriptor is
+ * a DEVICE pointer owned by the caller; the library allocates, frees and
+ * synchronises nothing (except pkv_device_error_flags, which is documented
+ * as synchronous).  Every tensor pointer must be 16-byte aligned.  Calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ * stream).
+ *
+ * Errors: each call returns PKV_OK (0) or a negative pkv_status.  Argument
+ * errors are found on the host before anything is launched.  PKV_ERR_CUDA
+ * reports a failed launch.  Values that live in device memory (page ids,
+ * lengths, slots) cannot be checked on the host; kernels check the ones that
+ * would make them read or write outside the arrays given, skip that work,
+ * and raise a bit in a device-side error word that pkv_device_error_flags
+ * returns.  No kernel traps.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle as cudaStream_t, declared here so this header needs no CUDA
+ * headers. */
+typedef struct CUstream_st* pkv_stream_t;
+
+typedef struct {
+  int32_t num_pages;    /* pages in each pool */
+  int32_t page_size;    /* P: token rows per page (16 or 32) */
+  int32_t num_kv_heads; /* Hkv */
+  int32_t head_dim;     /* d (64 or 128) */
+} pkv_pool_desc;
+
+enum pkv_status {
+  PKV_OK = 0,
+  PKV_ERR_NULL_POINTER = -1,  /* a required pointer is NULL */
+  PKV_ERR_BAD_SHAPE = -2,     /* negative size, Hq % Hkv != 0, ... */
+  PKV_ERR_UNSUPPORTED = -3,   /* head_dim, page_size or group size outside the supported set */
+  PKV_ERR_MISALIGNED = -4,    /* a tensor pointer is not 16-byte aligned */
+  PKV_ERR_WORKSPACE = -5,     /* workspace NULL or smaller than required */
+  PKV_ERR_CUDA = -6,          /* a CUDA launch or runtime call failed */
+  PKV_ERR_DEVICE = -7,        /* current device is not sm_100 */
+  PKV_ERR_TENSOR_MAP = -8     /* the driver rejected a TMA tensor map */
+};
+
+/* Bits of the device-side error word (see pkv_device_error_flags). */
+#define PKV_FLAG_WAIT_TIMEOUT   0x1u  /* a pipeline wait hit its ~2 s limit; the kernel gave up */
+#define PKV_FLAG_BAD_LENGTH     0x2u  /* a kv_len/ctx/chunk length < 0 or beyond max_pages*page_size */
+#define PKV_FLAG_BAD_SLOT       0x4u  /* kv_append slot >= num_pages*page_size (row skipped) */
+#define PKV_FLAG_BAD_QUERY_ROWS 0x8u  /* cu_q_lens not non-decreasing within [0, total_q] */
+#define PKV_FLAG_BAD_PAGE       0x10u /* a page-table entry outside [0, num_pages) was read (as zeros) */
+
+/*
+ * pkv_kv_append -- write the K/V rows of this step's new tokens into pool
+ * pages through a slot mapping (on-demand pages of the tiny-llm source
+ * reading, "Paged KV Cache"; the slot mapping is the batch's dynamic slot ->
+ * request map of its TinyLlmBatch, "Continuous Batching").
+ *
+ *   k_new, v_new   [num_tokens][Hkv][d] bf16
+ *   slot_mapping   [num_tokens] int32; row t goes to slot slot_mapping[t] of
+ *                  both pools; -1 skips the row (padding)
+ *   k_pool, v_pool pools as above, written in place
+ *
+ * A pure bit copy: each pool row equals its source row bit for bit.  Slots
+ * beyond the pool raise PKV_FLAG_BAD_SLOT and are skipped.  Two rows with the
+ * same slot race (one of them wins).  num_tokens == 0 launches nothing.
+ */
+PKV_API int pkv_kv_append(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                  int32_t num_tokens, void* k_pool, void* v_pool, pkv_pool_desc pool,
+                  pkv_stream_t stream);
+
+/*
+ * pkv_decode_workspace_bytes -- bytes of workspace pkv_paged_attn_decode
+ * needs for `batch` requests whose lengths are at most max_kv_len (pass
+ * max_pages * page_size).  partition_tokens as in pkv_paged_attn_decode.
+ */
+PKV_API size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                  int32_t max_kv_len, int32_t partition_tokens);
+
+/*
+ * pkv_paged_attn_decode -- q_len = 1 attention of each request over its whole
+ * paged context (paged FlashAttention, decode).  One KV read serves all query
+ * heads of a GQA group.  Long contexts are cut into split-K partitions
+ * (flash-decoding) whose partials are merged by pkv_split_k_combine's rule.
+ *
+ *   q           [batch][Hq][d] bf16; request r's query sits at position
+ *               kv_lens[r] - 1
+ *   page_table  [batch][max_pages] int32
+ *   kv_lens     [batch] int32, keys per request INCLUDING the token appended
+ *               this step; 0 gives a zero output (lse -inf)
+ *   scale       softmax scale (usually 1/sqrt(d))
+ *   partition_tokens  split-K partition length in tokens: 0 = chosen on the
+ *               device from the lengths and the SM count; -1 = never split;
+ *               otherwise a multiple of 32 in [32, 65536]
+ *   workspace   device scratch of pkv_decode_workspace_bytes(...) bytes,
+ *               holding split partials and two scheduling counters.  It must
+ *               be ZERO-FILLED before its first use; every call leaves the
+ *               counters at zero again.  Calls that share a workspace must
+ *               not overlap in time.
+ *   out         [batch][Hq][d] bf16 (written)
+ *   out_lse     [batch][Hq] fp32 natural-log softmax denominators, or NULL
+ *
+ * Requests whose length fits one partition are written by the partition
+ * kernel directly; the others go through partials and the combine kernel.
+ */
+PKV_API int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads,
+                          const void* k_pool, const void* v_pool, pkv_pool_desc pool,
+                          const int32_t* page_table, int32_t max_pages,
+                          const int32_t* kv_lens, float scale, int32_t partition_tokens,
+                          void* workspace, size_t workspace_bytes, void* out,
+                          float* out_lse, pkv_stream_t stream);
+
+/*
+ * pkv_split_k_combine -- merge split-K partials by their log-sum-exp weights
+ * (mini-vllm advanced series design, adv04 "Flash-Decoding"; the formula is
+ * the plain reading: M = max_s lse_s, w_s = exp(lse_s - M),
+ * o = sum_s w_s o_s / sum_s w_s, lse = M + ln sum_s w_s).
+ *
+ *   part_o      [batch][Hq][max_splits][d] fp32, each partial normalised
+ *               within its split
+ *   part_lse    [batch][Hq][max_splits] fp32 natural-log denominators;
+ *               -inf marks an empty split (weight 0)
+ *   num_splits  [batch] int32, splits used by each request (<= max_splits)
+ *   out         [batch][Hq][d] bf16; out_lse [batch][Hq] fp32 or NULL
+ *
+ * A request with no non-empty split gets a zero output and lse -inf.
+ */
+PKV_API int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
+                        int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                        int32_t max_splits, void* out, float* out_lse, pkv_stream_t stream);
+
+/*
+ * pkv_paged_attn_chunked_prefill -- causal attention of prompt chunks at
+ * per-request context offsets, on tensor cores (tcgen05, TMEM accumulators),
+ * reading keys from the paged pool (tiny-llm source reading, "Chunked
+ * Prefill": a long prompt is cut into bounded chunks interleaved with decode
+ * steps of other requests).
+ *
+ *   q            [total_q][Hq][d] bf16: request r's chunk is rows
+ *                cu_q_lens[r] .. cu_q_lens[r+1]-1
+ *   cu_q_lens    [batch+1] int32, non-decreasing, cu_q_lens[0] = 0,
+ *                cu_q_lens[batch] <= total_q
+ *   max_q_len    an upper bound on any chunk length (sizes the grid)
+ *   ctx_offsets  [batch] int32: tokens of request r before its chunk; chunk
+ *                row i sits at position ctx_offsets[r] + i and sees keys
+ *                0 .. ctx_offsets[r] + i (diagonal included)
+ *   page_table   [batch][max_pages] int32; the chunk's own K/V rows must
+ *                already be in the pool (pkv_kv_append first)
+ *   out          [total_q][Hq][d] bf16; rows past cu_q_lens[batch] are left
+ *                untouched
+ */
+PKV_API int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch,
+                                   int32_t num_q_heads, int32_t total_q, int32_t max_q_len,
+                                   const int32_t* ctx_offsets, const void* k_pool,
+                                   const void* v_pool, pkv_pool_desc pool,
+                                   const int32_t* page_table, int32_t max_pages, float scale,
+                                   void* out, pkv_stream_t stream);
+
+/* Human-readable name of a pkv_status value (static string). */
+PKV_API const char* pkv_status_string(int status);
+
+/*
+ * pkv_device_error_flags -- SYNCHRONOUS: waits for the current device, then
+ * returns the device-side error word (PKV_FLAG_* bits raised by any kernel of
+ * this library since the last clear) in *flags, and clears it when `clear`
+ * is nonzero.
+ */
+PKV_API int pkv_device_error_flags(uint32_t* flags, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,223 @@
+"""Paged KV-cache attention for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libpkv.so``, whose C ABI is declared in
+``include/pkv.h``.  Each function here has the name of the C entry point it
+calls and only marshals arguments: it checks dtypes and devices, passes raw
+device pointers, the current CUDA stream and the pool geometry, and turns a
+non-zero status into ``PkvError``.  All computation runs in the library's
+CUDA kernels; there is no CPU or PyTorch fallback, and importing this module
+fails if the library has not been built
+(``python paged_kv_attention_37_b200/build.py``).
+
+Tensors (all CUDA, contiguous):
+  k_pool, v_pool  bf16 [num_pages, Hkv, page_size, d]
+  page_table      int32 [B, max_pages]
+  kv_lens         int32 [B]      keys per request, including this step's token
+  q (decode)      bf16 [B, Hq, d]
+  q (prefill)     bf16 [total_q, Hq, d] with cu_q_lens int32 [B+1]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "PkvError", "LIB_PATH", "pool_desc", "pkv_kv_append", "pkv_decode_workspace_bytes",
+    "pkv_paged_attn_decode", "pkv_split_k_combine", "pkv_paged_attn_chunked_prefill",
+    "pkv_status_string", "pkv_device_error_flags", "decode_workspace",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
+
+FLAG_WAIT_TIMEOUT = 0x1
+FLAG_BAD_LENGTH = 0x2
+FLAG_BAD_SLOT = 0x4
+FLAG_BAD_QUERY_ROWS = 0x8
+FLAG_BAD_PAGE = 0x10
+
+
+class PkvError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {pkv_status_string(status)} (status {status})")
+        self.status = status
+
+
+class _PoolDesc(ctypes.Structure):
+    _fields_ = [("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "`python paged_kv_attention_37_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, SZ, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+    lib.pkv_kv_append.argtypes = [P, P, P, I32, P, P, _PoolDesc, P]
+    lib.pkv_kv_append.restype = ctypes.c_int
+    lib.pkv_decode_workspace_bytes.argtypes = [I32, I32, I32, I32, I32]
+    lib.pkv_decode_workspace_bytes.restype = SZ
+    lib.pkv_paged_attn_decode.argtypes = [P, I32, I32, P, P, _PoolDesc, P, I32, P, F32, I32, P, SZ,
+                                          P, P, P]
+    lib.pkv_paged_attn_decode.restype = ctypes.c_int
+    lib.pkv_split_k_combine.argtypes = [P, P, P, I32, I32, I32, I32, P, P, P]
+    lib.pkv_split_k_combine.restype = ctypes.c_int
+    lib.pkv_paged_attn_chunked_prefill.argtypes = [P, P, I32, I32, I32, I32, P, P, P, _PoolDesc, P,
+                                                   I32, F32, P, P]
+    lib.pkv_paged_attn_chunked_prefill.restype = ctypes.c_int
+    lib.pkv_status_string.argtypes = [ctypes.c_int]
+    lib.pkv_status_string.restype = ctypes.c_char_p
+    lib.pkv_device_error_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
+    lib.pkv_device_error_flags.restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+
+# ------------------------------------------------------------- marshalling
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int | None = None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise PkvError(fn, status)
+
+
+def pool_desc(k_pool: torch.Tensor) -> _PoolDesc:
+    n, hkv, p, d = k_pool.shape
+    return _PoolDesc(n, p, hkv, d)
+
+
+# -------------------------------------------------------------- entry points
+def pkv_status_string(status: int) -> str:
+    return _lib.pkv_status_string(int(status)).decode()
+
+
+def pkv_device_error_flags(clear: bool = True) -> int:
+    """Synchronise the device and return (and by default clear) the error word."""
+    v = ctypes.c_uint32(0)
+    _check("pkv_device_error_flags", _lib.pkv_device_error_flags(ctypes.byref(v), int(clear)))
+    return int(v.value)
+
+
+def pkv_kv_append(k_new, v_new, slot_mapping, k_pool, v_pool, stream=None):
+    """Bit-copy rows k_new/v_new [T, Hkv, d] into pool slots (slot = page*P + offset)."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _need(t, n, torch.bfloat16, 3)
+    _need(slot_mapping, "slot_mapping", torch.int32, 1)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    T = k_new.shape[0]
+    if slot_mapping.shape[0] != T or v_new.shape != k_new.shape:
+        raise ValueError("k_new, v_new and slot_mapping disagree on the token count")
+    if k_new.shape[1:] != (k_pool.shape[1], k_pool.shape[3]) or v_pool.shape != k_pool.shape:
+        raise ValueError("row shape does not match the pool")
+    _check("pkv_kv_append", _lib.pkv_kv_append(
+        _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(k_pool), _ptr(v_pool),
+        pool_desc(k_pool), _stream(stream)))
+
+
+def pkv_decode_workspace_bytes(batch, num_q_heads, head_dim, max_kv_len, partition_tokens=0) -> int:
+    return int(_lib.pkv_decode_workspace_bytes(batch, num_q_heads, head_dim, max_kv_len,
+                                               partition_tokens))
+
+
+def decode_workspace(batch, num_q_heads, head_dim, max_kv_len, partition_tokens=0, device=None):
+    """A zero-filled workspace of the size pkv_paged_attn_decode needs."""
+    n = pkv_decode_workspace_bytes(batch, num_q_heads, head_dim, max_kv_len, partition_tokens)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def pkv_paged_attn_decode(q, k_pool, v_pool, page_table, kv_lens, scale, partition_tokens=0,
+                          workspace=None, out=None, out_lse=None, stream=None):
+    """Decode attention (q_len = 1) of q [B, Hq, d] over each request's pages.
+
+    Returns ``out`` (bf16 [B, Hq, d]); fills ``out_lse`` (fp32 [B, Hq]) if given.
+    ``workspace`` (uint8, zero-filled before first use) defaults to a new one.
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    _need(page_table, "page_table", torch.int32, 2)
+    _need(kv_lens, "kv_lens", torch.int32, 1)
+    B, hq, d = q.shape
+    max_pages = page_table.shape[1]
+    if page_table.shape[0] != B or kv_lens.shape[0] != B:
+        raise ValueError("page_table / kv_lens rows must equal the batch")
+    if workspace is None:
+        workspace = decode_workspace(B, hq, d, max_pages * k_pool.shape[2], partition_tokens,
+                                     q.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 3)
+    if out_lse is not None:
+        _need(out_lse, "out_lse", torch.float32, 2)
+    _check("pkv_paged_attn_decode", _lib.pkv_paged_attn_decode(
+        _ptr(q), B, hq, _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table),
+        max_pages, _ptr(kv_lens), float(scale), int(partition_tokens), _ptr(workspace),
+        workspace.numel(), _ptr(out), _ptr(out_lse), _stream(stream)))
+    return out
+
+
+def pkv_split_k_combine(part_o, part_lse, num_splits, out=None, out_lse=None, stream=None):
+    """Merge fp32 partials part_o [B, Hq, S, d] / part_lse [B, Hq, S] -> bf16 [B, Hq, d]."""
+    _need(part_o, "part_o", torch.float32, 4)
+    _need(part_lse, "part_lse", torch.float32, 3)
+    _need(num_splits, "num_splits", torch.int32, 1)
+    B, hq, S, d = part_o.shape
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.bfloat16, device=part_o.device)
+    _need(out, "out", torch.bfloat16, 3)
+    if out_lse is not None:
+        _need(out_lse, "out_lse", torch.float32, 2)
+    _check("pkv_split_k_combine", _lib.pkv_split_k_combine(
+        _ptr(part_o), _ptr(part_lse), _ptr(num_splits), B, hq, d, S, _ptr(out), _ptr(out_lse),
+        _stream(stream)))
+    return out
+
+
+def pkv_paged_attn_chunked_prefill(q, cu_q_lens, ctx_offsets, k_pool, v_pool, page_table, scale,
+                                   max_q_len, out=None, stream=None):
+    """Causal attention of prompt chunks q [total_q, Hq, d] at context offsets."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(cu_q_lens, "cu_q_lens", torch.int32, 1)
+    _need(ctx_offsets, "ctx_offsets", torch.int32, 1)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    _need(page_table, "page_table", torch.int32, 2)
+    total_q, hq, d = q.shape
+    B = ctx_offsets.shape[0]
+    if cu_q_lens.shape[0] != B + 1 or page_table.shape[0] != B:
+        raise ValueError("cu_q_lens must have B+1 entries and page_table B rows")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 3)
+    _check("pkv_paged_attn_chunked_prefill", _lib.pkv_paged_attn_chunked_prefill(
+        _ptr(q), _ptr(cu_q_lens), B, hq, total_q, int(max_q_len), _ptr(ctx_offsets),
+        _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table), page_table.shape[1],
+        float(scale), _ptr(out), _stream(stream)))
+    return out

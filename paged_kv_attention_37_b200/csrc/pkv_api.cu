@@ -1,0 +1,394 @@
+// pkv_api.cu -- the C ABI declared in include/pkv.h: argument checks on the
+// host, TMA tensor maps, kernel selection by (head_dim, group size), and
+// launches.  The library allocates nothing and never synchronises the device
+// (pkv_device_error_flags excepted, as documented).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "decode.cuh"
+#include "kv_append.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+using pkv::decode::kChunk;
+
+struct DeviceInfo {
+  int sm_count = 0;
+  int major = 0, minor = 0;
+  bool valid = false;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+int current_device(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.valid) {
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return PKV_ERR_CUDA;
+    d.valid = true;
+  }
+  *out = d;
+  return (d.major == 10 && d.minor == 0) ? PKV_OK : PKV_ERR_DEVICE;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map: dims[0] innermost (elements), strides in bytes of
+// dims 1 and 2.
+int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+             uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2,
+             bool swizzle128) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return PKV_ERR_TENSOR_MAP;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1, stride2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_TENSOR_MAP;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_pool(const pkv_pool_desc& pool) {
+  if (pool.num_pages <= 0 || pool.num_kv_heads <= 0) return PKV_ERR_BAD_SHAPE;
+  if (pool.head_dim != 64 && pool.head_dim != 128) return PKV_ERR_UNSUPPORTED;
+  if (pool.page_size != 16 && pool.page_size != 32) return PKV_ERR_UNSUPPORTED;
+  // TMA row coordinate is page * Hkv + head, an int32
+  if (static_cast<long long>(pool.num_pages) * pool.num_kv_heads >= (1ll << 31)) return PKV_ERR_BAD_SHAPE;
+  return PKV_OK;
+}
+
+int check_heads(int32_t num_q_heads, const pkv_pool_desc& pool, int* group) {
+  if (num_q_heads <= 0 || num_q_heads % pool.num_kv_heads != 0) return PKV_ERR_BAD_SHAPE;
+  const int g = num_q_heads / pool.num_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return PKV_ERR_UNSUPPORTED;
+  *group = g;
+  return PKV_OK;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int32_t max_splits_for(int32_t max_kv_len, int32_t partition_tokens) {
+  if (partition_tokens < 0) return 1;
+  const int32_t part = partition_tokens > 0 ? partition_tokens : pkv::decode::kMinAutoPartition;
+  return std::max<int32_t>(1, (std::max<int32_t>(max_kv_len, 1) + part - 1) / part);
+}
+
+struct WorkspaceLayout {
+  size_t counters = 0, num_splits = 0, part_lse = 0, part_o = 0, total = 0;
+};
+
+WorkspaceLayout workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t S) {
+  WorkspaceLayout w;
+  w.counters = 0;
+  w.num_splits = 256;
+  w.part_lse = w.num_splits + align256(static_cast<size_t>(B) * 4);
+  w.part_o = w.part_lse + align256(static_cast<size_t>(B) * Hq * S * 4);
+  w.total = w.part_o + align256(static_cast<size_t>(B) * Hq * S * D * 4);
+  return w;
+}
+
+// ------------------------------------------------------------ decode launch
+template <int D, int G>
+int launch_decode(const pkv::decode::Params& prm, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                  int sm_count, cudaStream_t stream) {
+  constexpr int STAGES = D == 128 ? 4 : 8;
+  using LY = pkv::decode::Layout<D, G, STAGES>;
+  auto kernel = pkv::decode::partition_kernel<D, G, STAGES>;
+  const size_t smem = LY::bytes(prm.B);
+  if (smem > 227 * 1024) return PKV_ERR_BAD_SHAPE;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return PKV_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, pkv::decode::kThreads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return PKV_ERR_CUDA;
+  kernel<<<sm_count * per_sm, pkv::decode::kThreads, smem, stream>>>(kmap, vmap, prm);
+  if (launch_status() != PKV_OK) return PKV_ERR_CUDA;
+  const long long rows = static_cast<long long>(prm.B) * prm.Hq;
+  if (prm.partition >= 0) {  // with partition -1 every request is one split
+    const int blocks = static_cast<int>((rows + 3) / 4);
+    pkv::decode::combine_kernel<D><<<blocks, 128, 0, stream>>>(
+        prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.S_max, prm.out, prm.out_lse, 1);
+  }
+  return launch_status();
+}
+
+template <int D>
+int dispatch_decode_group(int group, const pkv::decode::Params& prm, const CUtensorMap& kmap,
+                          const CUtensorMap& vmap, int sm_count, cudaStream_t stream) {
+  switch (group) {
+    case 1: return launch_decode<D, 1>(prm, kmap, vmap, sm_count, stream);
+    case 2: return launch_decode<D, 2>(prm, kmap, vmap, sm_count, stream);
+    case 4: return launch_decode<D, 4>(prm, kmap, vmap, sm_count, stream);
+    case 8: return launch_decode<D, 8>(prm, kmap, vmap, sm_count, stream);
+  }
+  return PKV_ERR_UNSUPPORTED;
+}
+
+// ----------------------------------------------------------- prefill launch
+template <int D, int G>
+int launch_prefill(const pkv::prefill::Params& prm, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                   const CUtensorMap& vmap, int32_t max_q_len, cudaStream_t stream) {
+  using LY = pkv::prefill::Layout<D>;
+  auto kernel = pkv::prefill::prefill_kernel<D, G>;
+  // at least ~116 KB so that one CTA (and its 512 TMEM columns) owns an SM
+  const size_t smem = std::max<size_t>(LY::kBytes, 116 * 1024);
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return PKV_ERR_CUDA;
+  constexpr int QPOS = pkv::prefill::kM / G;
+  const long long tiles = (static_cast<long long>(max_q_len) + QPOS - 1) / QPOS;
+  const long long blocks = tiles * prm.Hkv * prm.B;
+  if (blocks == 0) return PKV_OK;
+  if (blocks > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
+  kernel<<<static_cast<unsigned>(blocks), pkv::prefill::kThreads, smem, stream>>>(qmap, kmap, vmap, prm);
+  return launch_status();
+}
+
+template <int D>
+int dispatch_prefill_group(int group, const pkv::prefill::Params& prm, const CUtensorMap& qmap,
+                           const CUtensorMap& kmap, const CUtensorMap& vmap, int32_t max_q_len,
+                           cudaStream_t stream) {
+  switch (group) {
+    case 1: return launch_prefill<D, 1>(prm, qmap, kmap, vmap, max_q_len, stream);
+    case 2: return launch_prefill<D, 2>(prm, qmap, kmap, vmap, max_q_len, stream);
+    case 4: return launch_prefill<D, 4>(prm, qmap, kmap, vmap, max_q_len, stream);
+    case 8: return launch_prefill<D, 8>(prm, qmap, kmap, vmap, max_q_len, stream);
+  }
+  return PKV_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pkv_status_string(int status) {
+  switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_NULL_POINTER: return "null pointer argument";
+    case PKV_ERR_BAD_SHAPE: return "invalid shape or size";
+    case PKV_ERR_UNSUPPORTED: return "unsupported head_dim, page_size or GQA group size";
+    case PKV_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case PKV_ERR_CUDA: return "CUDA launch or runtime error";
+    case PKV_ERR_DEVICE: return "current device is not sm_100 (B200)";
+    case PKV_ERR_TENSOR_MAP: return "TMA tensor map rejected by the driver";
+  }
+  return "unknown status";
+}
+
+int pkv_kv_append(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                  int32_t num_tokens, void* k_pool, void* v_pool, pkv_pool_desc pool,
+                  pkv_stream_t stream) {
+  if (num_tokens < 0) return PKV_ERR_BAD_SHAPE;
+  int st = check_pool(pool);
+  if (st != PKV_OK) return st;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool) return PKV_ERR_NULL_POINTER;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+    return PKV_ERR_MISALIGNED;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  const long long chunks = static_cast<long long>(num_tokens) * pool.num_kv_heads * (pool.head_dim / 8);
+  const int threads = 256;
+  const long long want = (chunks + threads - 1) / threads;
+  const int blocks = static_cast<int>(std::min<long long>(want, static_cast<long long>(dev.sm_count) * 16));
+  const int64_t num_slots = static_cast<int64_t>(pool.num_pages) * pool.page_size;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (pool.head_dim == 128)
+    pkv::kv_append_kernel<128><<<blocks, threads, 0, s>>>(
+        static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping, num_tokens,
+        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pool.num_kv_heads, pool.page_size, num_slots);
+  else
+    pkv::kv_append_kernel<64><<<blocks, threads, 0, s>>>(
+        static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping, num_tokens,
+        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pool.num_kv_heads, pool.page_size, num_slots);
+  return launch_status();
+}
+
+size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                  int32_t max_kv_len, int32_t partition_tokens) {
+  if (batch < 0 || num_q_heads < 0 || head_dim < 0 || max_kv_len < 0) return 0;
+  const int32_t S = max_splits_for(max_kv_len, partition_tokens);
+  return workspace_layout(batch, num_q_heads, head_dim, S).total;
+}
+
+int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool,
+                          const void* v_pool, pkv_pool_desc pool, const int32_t* page_table,
+                          int32_t max_pages, const int32_t* kv_lens, float scale,
+                          int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                          void* out, float* out_lse, pkv_stream_t stream) {
+  if (batch < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
+  int st = check_pool(pool);
+  if (st != PKV_OK) return st;
+  int group = 0;
+  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
+  if (partition_tokens > 0 && (partition_tokens % kChunk != 0 || partition_tokens > 65536))
+    return PKV_ERR_BAD_SHAPE;
+  if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
+  if (!std::isfinite(scale)) return PKV_ERR_BAD_SHAPE;
+  if (batch == 0) return PKV_OK;
+  if (!q || !k_pool || !v_pool || !page_table || !kv_lens || !out) return PKV_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return PKV_ERR_MISALIGNED;
+  const int32_t max_kv = max_pages * pool.page_size;
+  const int32_t S = max_splits_for(max_kv, partition_tokens);
+  const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, pool.head_dim, S);
+  if (workspace == nullptr || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  const int D = pool.head_dim;
+  const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
+  CUtensorMap kmap, vmap;
+  if ((st = make_map(&kmap, k_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
+                     pool.page_size, 1, true)) != PKV_OK)
+    return st;
+  if ((st = make_map(&vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, D,
+                     pool.page_size, 1, false)) != PKV_OK)
+    return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  pkv::decode::Params prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.page_table = page_table;
+  prm.kv_lens = kv_lens;
+  prm.out = static_cast<uint16_t*>(out);
+  prm.out_lse = out_lse;
+  prm.part_o = reinterpret_cast<float*>(ws + wl.part_o);
+  prm.part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
+  prm.num_splits = reinterpret_cast<int32_t*>(ws + wl.num_splits);
+  prm.counters = reinterpret_cast<uint32_t*>(ws + wl.counters);
+  prm.B = batch;
+  prm.Hq = num_q_heads;
+  prm.Hkv = pool.num_kv_heads;
+  prm.P = pool.page_size;
+  prm.max_pages = max_pages;
+  prm.num_pages = pool.num_pages;
+  prm.S_max = S;
+  prm.partition = partition_tokens;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 128) return dispatch_decode_group<128>(group, prm, kmap, vmap, dev.sm_count, s);
+  return dispatch_decode_group<64>(group, prm, kmap, vmap, dev.sm_count, s);
+}
+
+int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
+                        int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t max_splits,
+                        void* out, float* out_lse, pkv_stream_t stream) {
+  if (batch < 0 || num_q_heads <= 0 || max_splits <= 0) return PKV_ERR_BAD_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+  if (batch == 0) return PKV_OK;
+  if (!part_o || !part_lse || !num_splits || !out) return PKV_ERR_NULL_POINTER;
+  if (!aligned16(part_o) || !aligned16(out)) return PKV_ERR_MISALIGNED;
+  DeviceInfo dev;
+  int st;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  const long long rows = static_cast<long long>(batch) * num_q_heads;
+  const long long blocks = (rows + 3) / 4;
+  if (blocks > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (head_dim == 128)
+    pkv::decode::combine_kernel<128><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
+        part_o, part_lse, num_splits, batch, num_q_heads, max_splits, static_cast<uint16_t*>(out), out_lse, 0);
+  else
+    pkv::decode::combine_kernel<64><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
+        part_o, part_lse, num_splits, batch, num_q_heads, max_splits, static_cast<uint16_t*>(out), out_lse, 0);
+  return launch_status();
+}
+
+int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch,
+                                   int32_t num_q_heads, int32_t total_q, int32_t max_q_len,
+                                   const int32_t* ctx_offsets, const void* k_pool, const void* v_pool,
+                                   pkv_pool_desc pool, const int32_t* page_table, int32_t max_pages,
+                                   float scale, void* out, pkv_stream_t stream) {
+  if (batch < 0 || total_q < 0 || max_q_len < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
+  int st = check_pool(pool);
+  if (st != PKV_OK) return st;
+  int group = 0;
+  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
+  if (!std::isfinite(scale)) return PKV_ERR_BAD_SHAPE;
+  if (batch == 0 || total_q == 0 || max_q_len == 0) return PKV_OK;
+  if (!q || !cu_q_lens || !ctx_offsets || !k_pool || !v_pool || !page_table || !out)
+    return PKV_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return PKV_ERR_MISALIGNED;
+  if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  const int D = pool.head_dim;
+  const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
+  const int qpos = pkv::prefill::kM / group;
+  CUtensorMap qmap, kmap, vmap;
+  if ((st = make_map(&qmap, q, D, num_q_heads, total_q, D * 2ull, static_cast<uint64_t>(num_q_heads) * D * 2, 64,
+                     group, qpos, true)) != PKV_OK)
+    return st;
+  if ((st = make_map(&kmap, k_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
+                     pool.page_size, 1, true)) != PKV_OK)
+    return st;
+  if ((st = make_map(&vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
+                     pool.page_size, 1, true)) != PKV_OK)
+    return st;
+  pkv::prefill::Params prm;
+  prm.cu_q_lens = cu_q_lens;
+  prm.ctx_offsets = ctx_offsets;
+  prm.page_table = page_table;
+  prm.out = static_cast<uint16_t*>(out);
+  prm.B = batch;
+  prm.Hq = num_q_heads;
+  prm.Hkv = pool.num_kv_heads;
+  prm.P = pool.page_size;
+  prm.max_pages = max_pages;
+  prm.num_pages = pool.num_pages;
+  prm.total_q = total_q;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 128) return dispatch_prefill_group<128>(group, prm, qmap, kmap, vmap, max_q_len, s);
+  return dispatch_prefill_group<64>(group, prm, qmap, kmap, vmap, max_q_len, s);
+}
+
+int pkv_device_error_flags(uint32_t* flags, int clear) {
+  if (flags == nullptr) return PKV_ERR_NULL_POINTER;
+  if (cudaDeviceSynchronize() != cudaSuccess) return PKV_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, pkv::g_error_flags, sizeof(v)) != cudaSuccess) return PKV_ERR_CUDA;
+  *flags = v;
+  if (clear) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(pkv::g_error_flags, &zero, sizeof(zero)) != cudaSuccess) return PKV_ERR_CUDA;
+  }
+  return PKV_OK;
+}
+
+}  // extern "C"

@@ -290,7 +290,8 @@ def make_workload(name: str, seed: int = 0, **over) -> Workload:
     """Build one of the named workloads; keyword overrides shrink it for tests.
 
     Recognised overrides: B (batch), len_lo/len_hi (uniform lengths),
-    lens (explicit kv lengths), n_prefill/chunk/ctx_hi/n_decode (mixed batch),
+    lens (explicit kv lengths), n_prefill/chunk/chunks/ctx_hi/ctxs/n_decode
+    (mixed batch),
     median (lognormal median), max_len, page_size, num_q_heads, num_kv_heads,
     head_dim.
     """
@@ -319,6 +320,8 @@ def make_workload(name: str, seed: int = 0, **over) -> Workload:
         n_pre, chunk = over.get("n_prefill", 8), over.get("chunk", 512)
         n_dec = over.get("n_decode", 56)
         ctx_pre = rng.integers(0, over.get("ctx_hi", 8192), size=n_pre, endpoint=True)
+        if "ctxs" in over:
+            ctx_pre = np.asarray(over["ctxs"], dtype=np.int64)
         chunks = np.asarray(over.get("chunks", [chunk] * n_pre), dtype=np.int64)
         kv_dec = rng.integers(over.get("len_lo", 256), over.get("len_hi", 4096), size=n_dec, endpoint=True)
         ctx = np.concatenate([ctx_pre, kv_dec - 1]).astype(np.int32)
