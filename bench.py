@@ -360,7 +360,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workloads", default="all",
                     help="extra workloads to measure besides the headline: all, none, or a list")
-    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of CPU time for the oracle baseline; 0 skips it")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -414,7 +415,8 @@ def main():
             dist.barrier()
             dist.destroy_process_group()
         return 0
-    cpu_rate, cpu_secs, sample = cpu_oracle_rate(HEADLINE, args.cpu_budget) if world == 1 else (None, None, None)
+    cpu_rate, cpu_secs, sample = (cpu_oracle_rate(HEADLINE, args.cpu_budget)
+                                  if world == 1 and args.cpu_budget > 0 else (None, None, None))
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,

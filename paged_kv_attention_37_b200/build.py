@@ -31,8 +31,8 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found; set NVCC or put CUDA's bin directory on PATH")
 
 
-def command(out: str = LIB, ptxas_verbose: bool = False) -> list[str]:
-    cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
+def command(out: str = LIB, ptxas_verbose: bool = False, defines=()) -> list[str]:
+    cmd = [nvcc_path(), *[f"-D{d}" for d in defines], "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
            "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-shared", "--cudart", "static", "-o", out]
     if ptxas_verbose:

@@ -9,26 +9,30 @@
 // mini-vllm advanced series design, section 4 Phase B adv04 (split-K over a
 // long KV sequence).
 //
-// Work unit ("item"): one (request r, KV head g, split s) triple; it covers
-// tokens [s*part, min((s+1)*part, L_r)) and produces the outputs of all G
-// query heads of the group, so every K/V byte is read from HBM once and used
-// G times.  A persistent grid takes items from an atomic counter in the
-// workspace (dynamic load balancing over ragged lengths).
+// Work unit ("item"): one (request r, KV head g, split s); it covers tokens
+// [s*part, min((s+1)*part, L_r)) and produces the outputs of all G query
+// heads of the group, so every K/V byte is read from HBM once and used G
+// times.  Items whose length is a whole partition are handed out first, the
+// shorter remainders last (largest-first order), from an atomic counter in
+// the workspace (dynamic load balancing over ragged lengths).
 //
-// CTA layout: warp 0 is the producer, warps 1..4 are consumers.
-//   producer: walks the item's page-table entries (32 at a time, loaded by
-//     the whole warp), and for each 32-token chunk issues TMA tensor loads of
-//     the K block (128-byte swizzle) and V block of every page in the chunk
-//     into one ring stage, completing on that stage's mbarrier;
-//   consumers: chunk k of an item goes to consumer k % 4; a consumer keeps
-//     its own online-softmax state (running max m, per-lane partial sum l,
-//     output accumulator o) for the G heads; at the item's end the four
-//     states are merged through shared memory and written out: bf16 output
-//     when the request has one split, else an fp32 partial plus its lse.
-// Inside a chunk, lane t owns token t for the scores (q . k_t for G heads,
-// q read as broadcast fp32 from shared memory, k_t read from the swizzled
-// block without bank conflicts), and lane l owns output columns
-// [l*D/32, (l+1)*D/32) for P.V.
+// Every warp is independent: it takes an item, walks its page-table entries
+// (32 per warp-wide load), and keeps NS-1 chunks in flight in its own ring of
+// NS shared-memory stages of 8 KB: a chunk is 2048/d tokens (16 at d=128, 32
+// at d=64), fetched as TMA tensor boxes of 16 token rows -- K 128-byte
+// swizzled, V plain -- each box one page or half of a 32-token page,
+// completing on the stage's mbarrier, issued by lane 0 ahead of the chunk
+// being computed.  There is no cross-warp synchronisation after the planning
+// step, and the small per-warp footprint keeps 10-12 warps resident per SM.
+//
+// Inside a chunk every lane scores 64 elements of one token: at d=128 lanes
+// t and t+16 share token t (one half of d each, one shuffle adds them), at
+// d=64 lane t owns token t.  Scores use q as broadcast fp32 pairs from
+// shared memory (the halves padded onto different banks), k read from the
+// swizzled block without bank conflicts, and packed fp32x2 FMAs.  The online softmax keeps a warp-uniform
+// running max and per-lane partial sums.  For P.V lane l owns output columns
+// [l*D/32, (l+1)*D/32) of every head.  At the item's end the warp writes
+// bf16 output (single-split request) or an fp32 partial and its lse.
 #pragma once
 
 #include "ptx.cuh"
@@ -36,17 +40,22 @@
 namespace pkv {
 namespace decode {
 
-constexpr int kChunk = 32;       // tokens per pipeline stage
-constexpr int kConsumers = 4;    // consumer warps per CTA
-constexpr int kThreads = 32 * (kConsumers + 1);
-constexpr int kItemSlots = 8;    // ring of in-flight item descriptors
+constexpr int kBoxRows = 16;     // token rows per TMA box (a page, or half of one)
+template <int D>
+struct Chunk {
+  static constexpr int kLanesPerToken = D / 64;        // each lane scores 64 elements
+  static constexpr int kTokens = 32 / kLanesPerToken;  // tokens per pipeline stage
+  static constexpr int kBoxes = kTokens / kBoxRows;    // TMA boxes per stage (per K half)
+};
+constexpr int kItemSlots = 8;    // per-warp ring of item descriptors
 constexpr int kMinAutoPartition = 256;
 constexpr int kMaxAutoPartition = 8192;
-constexpr int kAutoItemsPerCta = 4;  // auto split: a CTA's share of work >= 4 partitions
+constexpr int kAutoItemsPerWarp = 3;  // auto split: each warp's share >= 3 partitions
 
-constexpr int kFlagLast = 1;  // this consumer's last stage of the item
-constexpr int kFlagDone = 2;  // no more items
-constexpr int kFlagQ = 4;     // stage also carries the item's G query rows
+constexpr int kPartitionQuantum = 32;  // split lengths are multiples of this
+constexpr float kLazyRescale = 8.0f;  // log2 units: move the running max when it grows > 2^8
+constexpr int kFirst = 1;  // first chunk of an item
+constexpr int kLast = 2;   // last chunk of an item
 
 struct Params {
   const uint16_t* q;          // bf16 [B][Hq][D]
@@ -57,34 +66,40 @@ struct Params {
   float* part_o;              // [B][Hq][S_max][D]
   float* part_lse;            // [B][Hq][S_max]
   int32_t* num_splits;        // [B]
-  uint32_t* counters;         // [0] next item, [1] finished CTAs
+  uint32_t* counters;         // [0] next item, [1] finished warps
   int32_t B, Hq, Hkv, P, max_pages, num_pages, S_max, partition;
   float scale_log2;           // softmax scale * log2(e)
 };
 
-struct StageInfo {
-  int32_t slot, ntok, flags, pad;
+struct ChunkInfo {
+  int32_t slot, ntok, flags, qslot;
 };
 struct ItemInfo {
   int32_t r, g, s, nsplit;
 };
 
-template <int D, int G, int STAGES>
+// Shared memory: one block per warp (the warp count W is chosen at launch
+// from the shared-memory budget), then the plan shared by the CTA.
+template <int D, int G, int NS>
 struct Layout {
-  static constexpr int kKBytes = kChunk * D * 2;  // [D/64][32 rows][128 B], swizzled
-  static constexpr int kVBytes = kChunk * D * 2;  // [32 rows][D] bf16
-  static constexpr int kQBytes = G * D * 2;       // [G][D] bf16
-  static constexpr int kStageBytes = (kKBytes + kVBytes + kQBytes + 1023) / 1024 * 1024;
-  static constexpr int kQfOff = STAGES * kStageBytes;                 // fp32 [NC][G][D]
-  static constexpr int kPbufOff = kQfOff + kConsumers * G * D * 4;    // fp32 [NC][32][G]
-  static constexpr int kMergeEntry = G * D + ((2 * G + 3) / 4) * 4;  // floats: o[G][D], m[G], l[G]
-  static constexpr int kMergeOff = kPbufOff + kConsumers * kChunk * G * 4;
-  static constexpr int kBarOff = kMergeOff + 2 * kConsumers * kMergeEntry * 4;
-  static constexpr int kInfoOff = kBarOff + (2 * STAGES + 2) * 8;
-  static constexpr int kItemOff = kInfoOff + STAGES * 16;
-  static constexpr int kMiscOff = kItemOff + kItemSlots * 16;
-  static constexpr int kLensOff = kMiscOff + 16;  // int32 lens[B], prefix[B+1]
-  static size_t bytes(int B) { return kLensOff + static_cast<size_t>(2 * B + 1) * 4 + 1024; }
+  static constexpr int kTok = Chunk<D>::kTokens;
+  static constexpr int kKBytes = kTok * D * 2;  // [D/64][kTok rows][128 B], swizzled
+  static constexpr int kVBytes = kTok * D * 2;  // [kTok rows][D] bf16
+  static constexpr int kStageBytes = kKBytes + kVBytes;
+  // scaled query pairs, fp32 [D/64 parts][32 pairs][G][2]; each part starts
+  // 16 bytes past a 128-byte multiple so the half-warps' broadcast reads land
+  // on different banks
+  static constexpr int kQHalfBytes = 32 * G * 8 + 16;
+  static constexpr int kQInOff = NS * kStageBytes;              // bf16 [NS][G][D] staged queries
+  static constexpr int kQfOff = kQInOff + NS * G * D * 2;
+  static constexpr int kPbOff = kQfOff + (D / 64) * kQHalfBytes;  // fp32 [kTok][G][2] (p, p) pairs
+  static constexpr int kBarOff = kPbOff + kTok * G * 8;         // NS mbarriers
+  static constexpr int kFifoOff = kBarOff + NS * 8;             // NS ChunkInfo
+  static constexpr int kItemOff = kFifoOff + NS * 16;           // kItemSlots ItemInfo
+  static constexpr int kWarpBytes = (kItemOff + kItemSlots * 16 + 1023) / 1024 * 1024;
+  // after the W warp blocks: misc[4], lens[B], prefF[B+1], prefR[B+1]
+  static size_t plan_bytes(int B) { return 16 + (3 * static_cast<size_t>(B) + 2) * 4; }
+  static size_t bytes(int W, int B) { return static_cast<size_t>(W) * kWarpBytes + plan_bytes(B) + 1024; }
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -107,42 +122,58 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-template <int D, int G, int STAGES>
-__global__ void __launch_bounds__(kThreads, 2) partition_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                             const __grid_constant__ CUtensorMap vmap,
-                                                             const Params p) {
-  using LY = Layout<D, G, STAGES>;
-  constexpr int DPL = D / 32;  // output columns per lane
+// largest r in [0, n) with pref[r] <= x (pref non-decreasing, pref[n] > x)
+__device__ __forceinline__ int upper_index(const int32_t* pref, int n, int x) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pref[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int D, int G, int NS, int MAXW>
+__global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                 const __grid_constant__ CUtensorMap vmap,
+                                                                 const Params p) {
+  using LY = Layout<D, G, NS>;
+  constexpr int kTok = Chunk<D>::kTokens, kLPT = Chunk<D>::kLanesPerToken;
+  const int W = blockDim.x >> 5;
+  const int log2P = 31 - __clz(p.P);  // P is a power of two
+  constexpr int DPL = D / 32;  // P.V output columns per lane
   static_assert(DPL == 2 || DPL == 4, "head_dim 64 or 128");
+  static_assert(NS >= 2, "at least two stages per warp");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const uint32_t sbase = smem_addr(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t* misc = reinterpret_cast<int32_t*>(smem + W * LY::kWarpBytes);
+  int32_t* lens = misc + 4;
+  int32_t* prefF = lens + p.B;
+  int32_t* prefR = prefF + p.B + 1;
 
-  auto full_bar = [&](int i) { return sbase + LY::kBarOff + 8u * i; };
-  auto empty_bar = [&](int i) { return sbase + LY::kBarOff + 8u * (STAGES + i); };
-  auto merge_bar = [&](int b) { return sbase + LY::kBarOff + 8u * (2 * STAGES + b); };
-  StageInfo* info = reinterpret_cast<StageInfo*>(smem + LY::kInfoOff);
-  ItemInfo* items = reinterpret_cast<ItemInfo*>(smem + LY::kItemOff);
-  int32_t* misc = reinterpret_cast<int32_t*>(smem + LY::kMiscOff);
-  int32_t* lens = reinterpret_cast<int32_t*>(smem + LY::kLensOff);
-  int32_t* prefix = lens + p.B;
+  uint8_t* wb = smem + warp * LY::kWarpBytes;
+  const uint32_t wbase = smem_addr(wb);
+  auto full_bar = [&](int i) { return wbase + LY::kBarOff + 8u * i; };
+  ChunkInfo* fifo = reinterpret_cast<ChunkInfo*>(wb + LY::kFifoOff);
+  ItemInfo* items = reinterpret_cast<ItemInfo*>(wb + LY::kItemOff);
+  float* qf = reinterpret_cast<float*>(wb + LY::kQfOff);
+  float* pb = reinterpret_cast<float*>(wb + LY::kPbOff);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(full_bar(i), 1);
-      mbar_init(empty_bar(i), 1);
-    }
-    mbar_init(merge_bar(0), kConsumers);
-    mbar_init(merge_bar(1), kConsumers);
+  if (lane == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(full_bar(i), 1);
     fence_barrier_init();
+  }
+  if (threadIdx.x == 0) {
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
   }
 
-  // ---- plan: clamp lengths, pick the partition, prefix-count the items
+  // ---- plan (warp 0): clamp lengths, pick the partition, count the items:
+  // whole-partition items first (prefF), then one remainder item per
+  // (request, KV head) whose length is not a multiple of the partition
+  // (prefR; an empty request also gets one, to write its zero output).
   if (warp == 0) {
     const int maxL = p.max_pages * p.P;
     long long tot = 0;
@@ -163,397 +194,450 @@ __global__ void __launch_bounds__(kThreads, 2) partition_kernel(const __grid_con
     if (p.partition > 0) {
       part = p.partition;
     } else if (p.partition < 0) {
-      part = ((maxL > 0 ? maxL : 1) + kChunk - 1) / kChunk * kChunk;
+      part = ((maxL > 0 ? maxL : 1) + kPartitionQuantum - 1) / kPartitionQuantum * kPartitionQuantum;
     } else {
-      const long long share = tot * p.Hkv / (static_cast<long long>(gridDim.x) * kAutoItemsPerCta);
+      const long long warps = static_cast<long long>(gridDim.x) * W;
+      const long long share = tot * p.Hkv / (warps * kAutoItemsPerWarp);
       part = kMaxAutoPartition;
       while (part > kMinAutoPartition && part > share) part >>= 1;
     }
     __syncwarp();
-    int running = 0;
+    int runF = 0, runR = 0;
     for (int base = 0; base < p.B; base += 32) {
       const int r = base + lane;
-      int ns = 0;
+      int nf = 0, nr = 0;
       if (r < p.B) {
         const int L = lens[r];
-        ns = L == 0 ? 1 : (L + part - 1) / part;
-        if (blockIdx.x == 0) p.num_splits[r] = ns;
+        nf = (L / part) * p.Hkv;
+        nr = (L % part != 0 || L == 0) ? p.Hkv : 0;
+        if (blockIdx.x == 0) p.num_splits[r] = L == 0 ? 1 : (L + part - 1) / part;
       }
-      int v = ns * p.Hkv;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += y;
+        const int yf = __shfl_up_sync(0xffffffffu, nf, o);
+        const int yr = __shfl_up_sync(0xffffffffu, nr, o);
+        if (lane >= o) {
+          nf += yf;
+          nr += yr;
+        }
       }
-      if (r < p.B) prefix[r + 1] = running + v;
-      running += __shfl_sync(0xffffffffu, v, 31);
+      if (r < p.B) {
+        prefF[r + 1] = runF + nf;
+        prefR[r + 1] = runR + nr;
+      }
+      runF += __shfl_sync(0xffffffffu, nf, 31);
+      runR += __shfl_sync(0xffffffffu, nr, 31);
     }
     if (lane == 0) {
-      prefix[0] = 0;
+      prefF[0] = 0;
+      prefR[0] = 0;
       misc[0] = part;
-      misc[1] = running;
+      misc[1] = runF;
+      misc[2] = runR;
     }
   }
   __syncthreads();
+  const int part = misc[0], nF = misc[1], total = misc[1] + misc[2];
 
-  if (warp == 0) {
-    // =========================== producer ===========================
-    const int part = misc[0], total_items = misc[1];
-    int seq = 0, item_count = 0;
-    bool ok = true;
-    while (ok) {
-      int item = 0;
-      if (lane == 0) item = static_cast<int>(atomicAdd(&p.counters[0], 1u));
-      item = __shfl_sync(0xffffffffu, item, 0);
-      if (item >= total_items) break;
-      int lo = 0, hi = p.B - 1;  // request r with prefix[r] <= item < prefix[r+1]
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (prefix[mid] <= item) lo = mid; else hi = mid - 1;
-      }
-      const int r = lo;
-      const int local = item - prefix[r];
-      const int s = local / p.Hkv, g = local - s * p.Hkv;
-      const int L = lens[r];
-      const int nsplit = L == 0 ? 1 : (L + part - 1) / part;
-      const int t0 = s * part, t1 = min(L, t0 + part);
-      const int ntok_item = max(0, t1 - t0);
-      const int nch = (ntok_item + kChunk - 1) / kChunk;
-      const int nst = max(1, (nch + kConsumers - 1) / kConsumers) * kConsumers;
-      const int slot = item_count % kItemSlots;
-      ++item_count;
-      if (lane == 0) items[slot] = ItemInfo{r, g, s, nsplit};
+  // ================= issue side: item cursor, lane 0 issues TMA =================
+  bool more = true, active = false;
+  int it_r = 0, it_g = 0, it_t0 = 0, it_ntok = 0, it_nch = 0, it_k = 0, it_slot = 0, it_qslot = 0;
+  int fetched = 0, pid_base = 0, pid_cur = -1, pid_next = -1, it_npg = 0;
+  const int32_t* ptab = p.page_table;
 
-      // page ids of this item, 32 entries per warp-wide load
-      const int npg = (ntok_item + p.P - 1) / p.P;
-      const int32_t* ptab = p.page_table + static_cast<size_t>(r) * p.max_pages + t0 / p.P;
-      int base = 0;
-      int pid_cur = lane < npg ? __ldg(ptab + lane) : -1;
-      int pid_next = 32 + lane < npg ? __ldg(ptab + 32 + lane) : -1;
-      const uint16_t* qsrc = p.q + (static_cast<size_t>(r) * p.Hq + static_cast<size_t>(g) * G) * D;
-
-      for (int k = 0; k < nst; ++k) {
-        const int stage = seq % STAGES;
-        if (seq >= STAGES && !mbar_wait(empty_bar(stage), ((seq / STAGES) - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        int flags = (k >= nst - kConsumers) ? kFlagLast : 0;
-        const uint32_t st = sbase + stage * LY::kStageBytes;
-        if (k < nch) {
-          const int tok0 = k * kChunk;  // relative to t0
-          const int ntok = min(kChunk, ntok_item - tok0);
-          const bool with_q = k < kConsumers;
-          if (with_q) flags |= kFlagQ;
-          const int npc = (ntok + p.P - 1) / p.P;  // pages touched by this chunk
-          int pids[kChunk / 16];
-#pragma unroll
-          for (int j = 0; j < kChunk / 16; ++j) {
-            pids[j] = -1;
-            if (j < npc) {
-              const int pi = tok0 / p.P + j;
-              while (pi >= base + 32) {
-                base += 32;
-                pid_cur = pid_next;
-                pid_next = base + 32 + lane < npg ? __ldg(ptab + base + 32 + lane) : -1;
-              }
-              pids[j] = __shfl_sync(0xffffffffu, pid_cur, pi & 31);
-            }
-          }
-          if (lane == 0) {
-            info[stage] = StageInfo{slot, ntok, flags, 0};
-            const uint32_t bytes = static_cast<uint32_t>(npc * p.P * D * 2 * 2) +
-                                   (with_q ? static_cast<uint32_t>(LY::kQBytes) : 0u);
-            mbar_arrive_expect_tx(full_bar(stage), bytes);
-#pragma unroll
-            for (int j = 0; j < kChunk / 16; ++j) {
-              if (j >= npc) break;
-              const int page = pids[j];
-              if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages))
-                raise_flag(PKV_FLAG_BAD_PAGE);  // TMA reads zeros out of bounds
-              const int row = page * p.Hkv + g;
-#pragma unroll
-              for (int h = 0; h < D / 64; ++h)
-                tma_load_3d(st + h * (kChunk * 128) + j * p.P * 128, &kmap, 64 * h, 0, row,
-                            full_bar(stage));
-              tma_load_3d(st + LY::kKBytes + j * p.P * D * 2, &vmap, 0, 0, row, full_bar(stage));
-            }
-            if (with_q) bulk_load(st + LY::kKBytes + LY::kVBytes, qsrc, LY::kQBytes, full_bar(stage));
-          }
-        } else if (lane == 0) {
-          info[stage] = StageInfo{slot, 0, flags, 0};
-          mbar_arrive(full_bar(stage));
-        }
-        __syncwarp();
-        ++seq;
-      }
+  auto fetch = [&]() {
+    int idx = 0;
+    if (lane == 0) idx = static_cast<int>(atomicAdd(p.counters, 1u));
+    idx = __shfl_sync(0xffffffffu, idx, 0);
+    if (idx >= total) {
+      more = false;
+      return;
     }
-    if (ok) {
-      for (int c = 0; c < kConsumers; ++c) {
-        const int stage = seq % STAGES;
-        if (seq >= STAGES && !mbar_wait(empty_bar(stage), ((seq / STAGES) - 1) & 1)) break;
-        if (lane == 0) {
-          info[stage] = StageInfo{0, 0, kFlagDone, 0};
-          mbar_arrive(full_bar(stage));
-        }
-        __syncwarp();
-        ++seq;
-      }
+    int r, g, s, t0, ntok;
+    if (idx < nF) {
+      r = upper_index(prefF, p.B, idx);
+      const int local = idx - prefF[r];
+      s = local / p.Hkv;
+      g = local - s * p.Hkv;
+      t0 = s * part;
+      ntok = part;
     } else {
-      // give copies already issued a bounded chance to land before exiting
-      for (int i = 0; i < STAGES && i < seq; ++i) {
-        const int sq = seq - 1 - i;
-        mbar_wait(full_bar(sq % STAGES), (sq / STAGES) & 1);
+      const int j = idx - nF;
+      r = upper_index(prefR, p.B, j);
+      g = j - prefR[r];
+      s = lens[r] / part;
+      t0 = s * part;
+      ntok = lens[r] - t0;
+    }
+    const int L = lens[r];
+    it_r = r;
+    it_g = g;
+    it_t0 = t0;
+    it_ntok = ntok;
+    it_nch = (ntok + kTok - 1) / kTok;
+    it_k = 0;
+    it_slot = fetched % kItemSlots;
+    it_qslot = fetched % NS;
+    ++fetched;
+    if (lane == 0) items[it_slot] = ItemInfo{r, g, s, L == 0 ? 1 : (L + part - 1) / part};
+    it_npg = (ntok + p.P - 1) >> log2P;
+    ptab = p.page_table + static_cast<size_t>(r) * p.max_pages + (t0 >> log2P);
+    pid_base = 0;
+    pid_cur = lane < it_npg ? __ldg(ptab + lane) : -1;
+    pid_next = 32 + lane < it_npg ? __ldg(ptab + 32 + lane) : -1;
+    active = true;
+  };
+
+  // Issue the next chunk of the current (or next) item into stage n % NS.
+  auto issue = [&](int n) -> bool {
+    if (!active) {
+      if (!more) return false;
+      fetch();
+      if (!active) return false;
+    }
+    const int stage = n % NS;
+    const int tok0 = it_k * kTok;  // relative to the item's first token (a page start)
+    const int ntok = it_nch == 0 ? 0 : min(kTok, it_ntok - tok0);
+    const int flags = (it_k == 0 ? kFirst : 0) | (it_k + 1 >= it_nch ? kLast : 0);
+    const int nbox = (ntok + kBoxRows - 1) / kBoxRows;
+    // each 16-row box lies inside one page: page-table entry (tok >> log2P),
+    // first row (tok & (P-1))
+    int pages[Chunk<D>::kBoxes];
+#pragma unroll
+    for (int b = 0; b < Chunk<D>::kBoxes; ++b) {
+      pages[b] = -1;
+      if (b < nbox) {
+        const int pi = (tok0 + b * kBoxRows) >> log2P;
+        while (pi >= pid_base + 32) {
+          pid_base += 32;
+          pid_cur = pid_next;
+          pid_next = pid_base + 32 + lane < it_npg ? __ldg(ptab + pid_base + 32 + lane) : -1;
+        }
+        pages[b] = __shfl_sync(0xffffffffu, pid_cur, pi & 31);
       }
     }
     if (lane == 0) {
-      __threadfence();
-      if (atomicAdd(&p.counters[1], 1u) == gridDim.x - 1) {
-        p.counters[0] = 0;
-        p.counters[1] = 0;
-        __threadfence();
+      fifo[stage] = ChunkInfo{it_slot, ntok, flags, it_qslot};
+      if (ntok > 0) {
+        const bool with_q = it_k == 0;
+        const uint32_t bytes = static_cast<uint32_t>(nbox * kBoxRows * D * 2 * 2) +
+                               (with_q ? static_cast<uint32_t>(G * D * 2) : 0u);
+        const uint32_t st = wbase + stage * LY::kStageBytes;
+        mbar_arrive_expect_tx(full_bar(stage), bytes);
+#pragma unroll
+        for (int b = 0; b < Chunk<D>::kBoxes; ++b) {
+          if (b >= nbox) break;
+          if (static_cast<unsigned>(pages[b]) >= static_cast<unsigned>(p.num_pages))
+            raise_flag(PKV_FLAG_BAD_PAGE);  // TMA reads zeros out of bounds
+          const int row = pages[b] * p.Hkv + it_g;
+          const int r0 = (tok0 + b * kBoxRows) & (p.P - 1);
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_3d(st + h * (kTok * 128) + b * (kBoxRows * 128), &kmap, 64 * h, r0, row,
+                        full_bar(stage));
+          tma_load_3d(st + LY::kKBytes + b * (kBoxRows * D * 2), &vmap, 0, r0, row, full_bar(stage));
+        }
+        if (with_q)
+          bulk_load(wbase + LY::kQInOff + it_qslot * (G * D * 2),
+                    p.q + (static_cast<size_t>(it_r) * p.Hq + static_cast<size_t>(it_g) * G) * D,
+                    G * D * 2, full_bar(stage));
+      } else {
+        mbar_arrive(full_bar(stage));
       }
     }
-    return;
-  }
+    __syncwarp();
+    if (++it_k >= max(1, it_nch)) active = false;
+    return true;
+  };
 
-  // ============================= consumers =============================
-  const int cw = warp - 1;
-  float* qf = reinterpret_cast<float*>(smem + LY::kQfOff) + cw * G * D;
-  float* pb = reinterpret_cast<float*>(smem + LY::kPbufOff) + cw * kChunk * G;
-  float* merge_base = reinterpret_cast<float*>(smem + LY::kMergeOff);
-  const uint32_t swz = static_cast<uint32_t>(lane & 7) << 4;
-
-  float o[G][DPL], m[G], l[G];
-  int seq = cw, cur_slot = -1, merged = 0;
-  while (true) {
-    const int stage = seq % STAGES;
-    if (!mbar_wait(full_bar(stage), (seq / STAGES) & 1)) break;
-    const StageInfo inf = info[stage];
-    if (inf.flags & kFlagDone) break;
-    const uint8_t* stp = smem + stage * LY::kStageBytes;
-    if (inf.slot != cur_slot) {
-      cur_slot = inf.slot;
+  // ================================ compute side ================================
+  // token of this lane, and which 64-element part of d it scores
+  const int tl = kLPT == 2 ? (lane & 15) : lane, hh = kLPT == 2 ? (lane >> 4) : 0;
+  const uint32_t swz = static_cast<uint32_t>(tl & 7) << 4;
+  float2 o2[G][DPL / 2];
+  float m[G], l[G];
+  int issued = 0;
+  while (issued < NS - 1 && issue(issued)) ++issued;
+  int n = 0;
+  for (; n < issued; ++n) {
+    const int stage = n % NS;
+    if (!mbar_wait(full_bar(stage), (n / NS) & 1)) break;
+    const ChunkInfo ci = fifo[stage];
+    const int ntok = ci.ntok;
+    if (ci.flags & kFirst) {
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         m[g] = -INFINITY;
         l[g] = 0.f;
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) o[g][e] = 0.f;
+        for (int e = 0; e < DPL / 2; ++e) o2[g][e] = make_float2(0.f, 0.f);
+      }
+      if (ntok > 0) {
+        // staged bf16 query rows [G][D] -> fp32 pairs [part][32][G][2],
+        // times scale*log2(e)
+        const uint32_t* qin = reinterpret_cast<const uint32_t*>(wb + LY::kQInOff + ci.qslot * (G * D * 2));
+        for (int i = lane; i < G * D / 2; i += 32) {
+          const int g = i / (D / 2), pp = i - g * (D / 2);
+          const int half = pp >> 5, ppl = pp & 31;
+          const uint32_t x = qin[i];
+          *reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(qf) + half * LY::kQHalfBytes + (ppl * G + g) * 8) =
+              make_float2(bf16lo(x) * p.scale_log2, bf16hi(x) * p.scale_log2);
+        }
       }
     }
-    if (inf.flags & kFlagQ) {
-      // query rows of the group -> fp32, pre-multiplied by scale*log2(e)
-      const uint16_t* qb = reinterpret_cast<const uint16_t*>(stp + LY::kKBytes + LY::kVBytes);
-      for (int i = lane * 2; i < G * D; i += 64) {
-        const uint32_t x = *reinterpret_cast<const uint32_t*>(qb + i);
-        qf[i] = bf16lo(x) * p.scale_log2;
-        qf[i + 1] = bf16hi(x) * p.scale_log2;
-      }
-      __syncwarp();
-    }
-    const int ntok = inf.ntok;
+    // keep NS-1 chunks in flight: refill the stage chunk n-1 used
+    __syncwarp();
+    fence_proxy_async_smem();
+    if (issue(issued)) ++issued;
+
     if (ntok > 0) {
-      // ---- scores: lane t <- token t
-      float acc[G];
+      const uint8_t* stp = wb + stage * LY::kStageBytes;
+      // ---- scores: each lane takes 64 elements (one 128-byte K row) of its token
+      float2 acc[G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = 0.f;
-      const uint8_t* krow = stp + lane * 128;
+      for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
+      const uint8_t* krow = stp + hh * (kTok * 128) + tl * 128;
+      const uint8_t* qh = reinterpret_cast<const uint8_t*>(qf) + hh * LY::kQHalfBytes;
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
+      for (int c = 0; c < 8; ++c) {
+        const uint4 kk = *reinterpret_cast<const uint4*>(krow + ((c << 4) ^ swz));
+        const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 kk =
-              *reinterpret_cast<const uint4*>(krow + h * (kChunk * 128) + ((c << 4) ^ swz));
-          const float k0 = bf16lo(kk.x), k1 = bf16hi(kk.x), k2 = bf16lo(kk.y), k3 = bf16hi(kk.y);
-          const float k4 = bf16lo(kk.z), k5 = bf16hi(kk.z), k6 = bf16lo(kk.w), k7 = bf16hi(kk.w);
+        for (int j = 0; j < 4; ++j) {
+          const float2 k2 = make_float2(bf16lo(kw[j]), bf16hi(kw[j]));
+          const int ppl = c * 4 + j;
+          if constexpr (G == 1) {
+            const float2 q2 = *reinterpret_cast<const float2*>(qh + ppl * 8);
+            acc[0] = __ffma2_rn(q2, k2, acc[0]);
+          } else {
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float4 qa = *reinterpret_cast<const float4*>(qf + g * D + h * 64 + c * 8);
-            const float4 qc = *reinterpret_cast<const float4*>(qf + g * D + h * 64 + c * 8 + 4);
-            float a = acc[g];
-            a = fmaf(qa.x, k0, a);
-            a = fmaf(qa.y, k1, a);
-            a = fmaf(qa.z, k2, a);
-            a = fmaf(qa.w, k3, a);
-            a = fmaf(qc.x, k4, a);
-            a = fmaf(qc.y, k5, a);
-            a = fmaf(qc.z, k6, a);
-            a = fmaf(qc.w, k7, a);
-            acc[g] = a;
+            for (int g = 0; g < G; g += 2) {
+              const float4 q4 = *reinterpret_cast<const float4*>(qh + (ppl * G + g) * 8);
+              acc[g] = __ffma2_rn(make_float2(q4.x, q4.y), k2, acc[g]);
+              acc[g + 1] = __ffma2_rn(make_float2(q4.z, q4.w), k2, acc[g + 1]);
+            }
           }
         }
       }
-      // ---- online softmax (log2 domain; hidden tokens get -inf -> weight 0)
+      // ---- online softmax, log2 domain; hidden tokens get -inf -> weight 0.
+      // The running max m is only moved (and o, l rescaled) when some score
+      // exceeds it by more than 2^8 -- in practice on an item's first chunk.
+      // Between moves the exponentials are taken against the stale max, so
+      // p <= 2^8; the final normalisation by l uses the same m, so the
+      // result is the same softmax.
+      float sv[G];
+      bool grow = false;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float sv = lane < ntok ? acc[g] : -INFINITY;
-        const float mn = fmaxf(m[g], warp_max(sv));
-        const float alpha = fast_exp2(m[g] - mn);
-        const float pv = fast_exp2(sv - mn);
-        l[g] = fmaf(l[g], alpha, pv);
+        float x = acc[g].x + acc[g].y;
+        if constexpr (kLPT == 2) x += __shfl_xor_sync(0xffffffffu, x, 16);
+        sv[g] = tl < ntok ? x : -INFINITY;
+        grow |= sv[g] > m[g] + kLazyRescale;
+      }
+      if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) o[g][e] *= alpha;
-        m[g] = mn;
-        pb[lane * G + g] = pv;
+        for (int g = 0; g < G; ++g) {
+          float mx = sv[g];
+#pragma unroll
+          for (int o = kTok / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float mn = fmaxf(m[g], mx);
+          const float alpha = fast_exp2(m[g] - mn);
+          l[g] *= alpha;
+          const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+          for (int e = 0; e < DPL / 2; ++e) o2[g][e] = __fmul2_rn(o2[g][e], a2);
+          m[g] = mn;
+        }
+      }
+      float pvs[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        pvs[g] = fast_exp2(sv[g] - m[g]);
+        if (hh == 0) l[g] += pvs[g];
+      }
+      if (hh == 0) {
+        if constexpr (G == 1) {
+          *reinterpret_cast<float2*>(pb + tl * 2) = make_float2(pvs[0], pvs[0]);
+        } else {
+#pragma unroll
+          for (int g = 0; g < G; g += 2)
+            *reinterpret_cast<float4*>(pb + (tl * G + g) * 2) = make_float4(pvs[g], pvs[g], pvs[g + 1], pvs[g + 1]);
+        }
       }
       __syncwarp();
-      // ---- P.V: lane owns DPL output columns
+      // ---- P.V: lane owns DPL output columns of every head
       const uint8_t* vb = stp + LY::kKBytes + lane * DPL * 2;
-#pragma unroll 4
-      for (int t = 0; t < ntok; ++t) {
-        float pg[G];
-        if constexpr (G % 4 == 0) {
-#pragma unroll
-          for (int g = 0; g < G; g += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(pb + t * G + g);
-            pg[g] = x.x; pg[g + 1] = x.y; pg[g + 2] = x.z; pg[g + 3] = x.w;
-          }
+      auto pv_token = [&](int t) {
+        float2 pg[G];
+        if constexpr (G == 1) {
+          pg[0] = *reinterpret_cast<const float2*>(pb + t * 2);
         } else {
 #pragma unroll
-          for (int g = 0; g < G; ++g) pg[g] = pb[t * G + g];
+          for (int g = 0; g < G; g += 2) {
+            const float4 x = *reinterpret_cast<const float4*>(pb + (t * G + g) * 2);
+            pg[g] = make_float2(x.x, x.y);
+            pg[g + 1] = make_float2(x.z, x.w);
+          }
         }
-        float v[DPL];
         if constexpr (DPL == 4) {
           const uint2 x = *reinterpret_cast<const uint2*>(vb + t * D * 2);
-          v[0] = bf16lo(x.x); v[1] = bf16hi(x.x); v[2] = bf16lo(x.y); v[3] = bf16hi(x.y);
+          const float2 v01 = make_float2(bf16lo(x.x), bf16hi(x.x));
+          const float2 v23 = make_float2(bf16lo(x.y), bf16hi(x.y));
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            o2[g][0] = __ffma2_rn(pg[g], v01, o2[g][0]);
+            o2[g][1] = __ffma2_rn(pg[g], v23, o2[g][1]);
+          }
         } else {
           const uint32_t x = *reinterpret_cast<const uint32_t*>(vb + t * D * 2);
-          v[0] = bf16lo(x); v[1] = bf16hi(x);
+          const float2 v01 = make_float2(bf16lo(x), bf16hi(x));
+#pragma unroll
+          for (int g = 0; g < G; ++g) o2[g][0] = __ffma2_rn(pg[g], v01, o2[g][0]);
         }
+      };
+      if (ntok == kTok) {  // full chunk: fully unrolled, constant offsets
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) o[g][e] = fmaf(pg[g], v[e], o[g][e]);
+        for (int t = 0; t < kTok; ++t) pv_token(t);
+      } else {
+#pragma unroll 1
+        for (int t = 0; t < ntok; ++t) pv_token(t);
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty_bar(stage));
 
-    if (inf.flags & kFlagLast) {
-      // ---- merge the four consumers' states of this item
-      const ItemInfo it = items[inf.slot];
-      const int b = merged & 1;
-      const uint32_t phase = (merged >> 1) & 1;
-      ++merged;
-      float* mine = merge_base + (b * kConsumers + cw) * LY::kMergeEntry;
+    if (ci.flags & kLast) {
+      // ---- item done: normalise and write bf16 output or an fp32 partial
+      const ItemInfo it = items[ci.slot];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float ls = warp_sum(l[g]);
-        if constexpr (DPL == 4) {
-          *reinterpret_cast<float4*>(mine + g * D + lane * 4) =
-              make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
-        } else {
-          *reinterpret_cast<float2*>(mine + g * D + lane * 2) = make_float2(o[g][0], o[g][1]);
-        }
-        if (lane == 0) {
-          mine[G * D + g] = m[g];
-          mine[G * D + G + g] = ls;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(merge_bar(b));
-      if (!mbar_wait(merge_bar(b), phase)) break;
-      const float* all = merge_base + b * kConsumers * LY::kMergeEntry;
-      for (int g = cw; g < G; g += kConsumers) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, all[w * LY::kMergeEntry + G * D + g]);
-        float den = 0.f, num[DPL];
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) num[e] = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-          for (int w = 0; w < kConsumers; ++w) {
-            const float* ew = all + w * LY::kMergeEntry;
-            const float f = fast_exp2(ew[G * D + g] - M);
-            den = fmaf(f, ew[G * D + G + g], den);
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) num[e] = fmaf(f, ew[g * D + lane * DPL + e], num[e]);
-          }
-        }
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        const float lse = den > 0.f ? (M + __log2f(den)) * 0.69314718055994531f : -INFINITY;
-        const int hq = it.g * G + g;
-        const size_t row = static_cast<size_t>(it.r) * p.Hq + hq;
+        const float inv = ls > 0.f ? 1.f / ls : 0.f;
+        const float lse = ls > 0.f ? (m[g] + __log2f(ls)) * 0.69314718055994531f : -INFINITY;
+        const size_t row = static_cast<size_t>(it.r) * p.Hq + it.g * G + g;
         if (it.nsplit == 1) {
           uint16_t* dst = p.out + row * D + lane * DPL;
           if constexpr (DPL == 4) {
             *reinterpret_cast<uint2*>(dst) =
-                make_uint2(pack_bf16x2(num[0] * inv, num[1] * inv), pack_bf16x2(num[2] * inv, num[3] * inv));
+                make_uint2(pack_bf16x2(o2[g][0].x * inv, o2[g][0].y * inv),
+                           pack_bf16x2(o2[g][1].x * inv, o2[g][1].y * inv));
           } else {
-            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(num[0] * inv, num[1] * inv);
+            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(o2[g][0].x * inv, o2[g][0].y * inv);
           }
           if (p.out_lse != nullptr && lane == 0) p.out_lse[row] = lse;
         } else {
           const size_t prow = row * p.S_max + it.s;
           float* dst = p.part_o + prow * D + lane * DPL;
           if constexpr (DPL == 4) {
-            *reinterpret_cast<float4*>(dst) =
-                make_float4(num[0] * inv, num[1] * inv, num[2] * inv, num[3] * inv);
+            *reinterpret_cast<float4*>(dst) = make_float4(o2[g][0].x * inv, o2[g][0].y * inv,
+                                                          o2[g][1].x * inv, o2[g][1].y * inv);
           } else {
-            *reinterpret_cast<float2*>(dst) = make_float2(num[0] * inv, num[1] * inv);
+            *reinterpret_cast<float2*>(dst) = make_float2(o2[g][0].x * inv, o2[g][0].y * inv);
           }
           if (lane == 0) p.part_lse[prow] = lse;
         }
       }
     }
-    seq += kConsumers;
+  }
+  if (n < issued) {
+    // a wait gave up: give copies still in flight a bounded chance to land
+    for (int k = n + 1; k < issued; ++k) mbar_wait(full_bar(k % NS), (k / NS) & 1);
+  }
+  if (lane == 0) {
+    __threadfence();
+    if (atomicAdd(&p.counters[1], 1u) == gridDim.x * W - 1) {
+      p.counters[0] = 0;
+      p.counters[1] = 0;
+      __threadfence();
+    }
   }
 }
 
-// Merge split partials.  One warp per (request, query head); lane owns D/32
-// columns.  skip_single: requests with one split were written by the
-// partition kernel already.
+// Merge split partials.  One CTA per (request, query head) row; its warps
+// stride over the splits (four splits' loads in flight per warp), each lane
+// owning D/32 columns, and the per-warp sums meet in shared memory.
+// skip_single: requests with one split were written by the partition kernel.
+constexpr int kCombineMaxWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part_o,
-                                                      const float* __restrict__ part_lse,
-                                                      const int32_t* __restrict__ num_splits,
-                                                      int32_t B, int32_t Hq, int32_t S_max,
-                                                      uint16_t* __restrict__ out,
-                                                      float* __restrict__ out_lse,
-                                                      int skip_single) {
+__global__ void __launch_bounds__(32 * kCombineMaxWarps) combine_kernel(
+    const float* __restrict__ part_o, const float* __restrict__ part_lse,
+    const int32_t* __restrict__ num_splits, int32_t B, int32_t Hq, int32_t S_max,
+    uint16_t* __restrict__ out, float* __restrict__ out_lse, int skip_single) {
   constexpr int DPL = D / 32;
   constexpr float kLog2e = 1.4426950408889634f;
-  const int lane = threadIdx.x & 31;
-  const long long idx = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
-  if (idx >= static_cast<long long>(B) * Hq) return;
-  const int r = static_cast<int>(idx / Hq);
+  __shared__ float red_m[kCombineMaxWarps], red_den[kCombineMaxWarps];
+  __shared__ __align__(16) float red_acc[kCombineMaxWarps][D];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const long long row = blockIdx.x;
+  const int r = static_cast<int>(row / Hq);
   int n = num_splits[r];
   if (skip_single && n <= 1) return;
   n = max(0, min(n, S_max));
-  const float* ls = part_lse + idx * S_max;
+  const float* ls = part_lse + row * S_max;
   float M = -INFINITY;
-  for (int s = lane; s < n; s += 32) M = fmaxf(M, ls[s]);
+  for (int s = threadIdx.x; s < n; s += blockDim.x) M = fmaxf(M, ls[s]);
   M = warp_max(M);
+  if (lane == 0) red_m[warp] = M;
+  __syncthreads();
+  M = red_m[0];
+  for (int w = 1; w < nw; ++w) M = fmaxf(M, red_m[w]);
   float acc[DPL], den = 0.f;
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
   if (M != -INFINITY) {
-    const float* po = part_o + idx * S_max * D + lane * DPL;
-#pragma unroll 4
-    for (int s = 0; s < n; ++s) {
-      const float w = fast_exp2((ls[s] - M) * kLog2e);
-      den += w;
+    const float* po = part_o + row * S_max * D + lane * DPL;
+    auto load = [&](int s, float (&v)[DPL]) {
       if constexpr (DPL == 4) {
         const float4 x = *reinterpret_cast<const float4*>(po + static_cast<size_t>(s) * D);
-        acc[0] = fmaf(w, x.x, acc[0]); acc[1] = fmaf(w, x.y, acc[1]);
-        acc[2] = fmaf(w, x.z, acc[2]); acc[3] = fmaf(w, x.w, acc[3]);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
       } else {
         const float2 x = *reinterpret_cast<const float2*>(po + static_cast<size_t>(s) * D);
-        acc[0] = fmaf(w, x.x, acc[0]); acc[1] = fmaf(w, x.y, acc[1]);
+        v[0] = x.x; v[1] = x.y;
+      }
+    };
+    int s = warp;
+    for (; s + 3 * nw < n; s += 4 * nw) {
+      float v[4][DPL], lv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        lv[u] = ls[s + u * nw];
+        load(s + u * nw, v[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = fast_exp2((lv[u] - M) * kLog2e);
+        den += w;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, v[u][e], acc[e]);
       }
     }
+    for (; s < n; s += nw) {
+      float v[DPL];
+      load(s, v);
+      const float w = fast_exp2((ls[s] - M) * kLog2e);
+      den += w;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, v[e], acc[e]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) red_acc[warp][lane * DPL + e] = acc[e];
+  if (lane == 0) red_den[warp] = den;
+  __syncthreads();
+  if (warp != 0) return;
+  for (int w = 1; w < nw; ++w) {
+    den += red_den[w];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] += red_acc[w][lane * DPL + e];
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  uint16_t* dst = out + idx * D + lane * DPL;
+  uint16_t* dst = out + row * D + lane * DPL;
   if constexpr (DPL == 4) {
     *reinterpret_cast<uint2*>(dst) =
         make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
   } else {
     *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }
-  if (out_lse != nullptr && lane == 0) out_lse[idx] = den > 0.f ? M + logf(den) : -INFINITY;
+  if (out_lse != nullptr && lane == 0) out_lse[row] = den > 0.f ? M + logf(den) : -INFINITY;
 }
 
 }  // namespace decode

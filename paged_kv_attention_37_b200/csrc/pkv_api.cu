@@ -15,7 +15,6 @@
 
 namespace {
 
-using pkv::decode::kChunk;
 
 struct DeviceInfo {
   int sm_count = 0;
@@ -95,6 +94,24 @@ int check_heads(int32_t num_q_heads, const pkv_pool_desc& pool, int* group) {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
 
+// warps per combine CTA: about one per eight splits, a power of two in [1, 8]
+int combine_warps(int32_t max_splits) {
+  int w = 1;
+  while (w < pkv::decode::kCombineMaxWarps && w * 8 < max_splits) w <<= 1;
+  return w;
+}
+
+template <int D>
+int launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits, int32_t B,
+                   int32_t Hq, int32_t S, uint16_t* out, float* out_lse, int skip_single,
+                   cudaStream_t stream) {
+  const long long rows = static_cast<long long>(B) * Hq;
+  if (rows > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
+  pkv::decode::combine_kernel<D><<<static_cast<unsigned>(rows), 32 * combine_warps(S), 0, stream>>>(
+      part_o, part_lse, num_splits, B, Hq, S, out, out_lse, skip_single);
+  return launch_status();
+}
+
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 int32_t max_splits_for(int32_t max_kv_len, int32_t partition_tokens) {
@@ -121,28 +138,35 @@ WorkspaceLayout workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t S) {
 template <int D, int G>
 int launch_decode(const pkv::decode::Params& prm, const CUtensorMap& kmap, const CUtensorMap& vmap,
                   int sm_count, cudaStream_t stream) {
-  constexpr int STAGES = D == 128 ? 4 : 8;
-  using LY = pkv::decode::Layout<D, G, STAGES>;
-  auto kernel = pkv::decode::partition_kernel<D, G, STAGES>;
-  const size_t smem = LY::bytes(prm.B);
-  if (smem > 227 * 1024) return PKV_ERR_BAD_SHAPE;
+#ifndef PKV_DECODE_NS128
+#define PKV_DECODE_NS128 2
+#endif
+#ifndef PKV_DECODE_NS64
+#define PKV_DECODE_NS64 3
+#endif
+#ifndef PKV_DECODE_MAXW128
+#define PKV_DECODE_MAXW128 10
+#endif
+#ifndef PKV_DECODE_MAXW64
+#define PKV_DECODE_MAXW64 12
+#endif
+  constexpr int NS = D == 128 ? PKV_DECODE_NS128 : PKV_DECODE_NS64;        // stages per warp
+  constexpr int kMaxW = D == 128 ? PKV_DECODE_MAXW128 : PKV_DECODE_MAXW64;  // warps per CTA
+  using LY = pkv::decode::Layout<D, G, NS>;
+  auto kernel = pkv::decode::partition_kernel<D, G, NS, kMaxW>;
+  constexpr size_t kBudget = 227 * 1024;
+  const size_t fixed = LY::plan_bytes(prm.B) + 1024;
+  if (fixed + LY::kWarpBytes > kBudget) return PKV_ERR_BAD_SHAPE;  // batch too large for the plan
+  const int W = static_cast<int>(std::min<size_t>(kMaxW, (kBudget - fixed) / LY::kWarpBytes));
+  const size_t smem = LY::bytes(W, prm.B);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return PKV_ERR_CUDA;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, pkv::decode::kThreads, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
-    return PKV_ERR_CUDA;
-  kernel<<<sm_count * per_sm, pkv::decode::kThreads, smem, stream>>>(kmap, vmap, prm);
+  kernel<<<sm_count, W * 32, smem, stream>>>(kmap, vmap, prm);
   if (launch_status() != PKV_OK) return PKV_ERR_CUDA;
-  const long long rows = static_cast<long long>(prm.B) * prm.Hq;
-  if (prm.partition >= 0) {  // with partition -1 every request is one split
-    const int blocks = static_cast<int>((rows + 3) / 4);
-    pkv::decode::combine_kernel<D><<<blocks, 128, 0, stream>>>(
-        prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.S_max, prm.out, prm.out_lse, 1);
-  }
-  return launch_status();
+  if (prm.partition < 0) return PKV_OK;  // every request is one split
+  return launch_combine<D>(prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.S_max, prm.out,
+                           prm.out_lse, 1, stream);
 }
 
 template <int D>
@@ -255,7 +279,8 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   if (st != PKV_OK) return st;
   int group = 0;
   if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
-  if (partition_tokens > 0 && (partition_tokens % kChunk != 0 || partition_tokens > 65536))
+  if (partition_tokens > 0 &&
+      (partition_tokens % pkv::decode::kPartitionQuantum != 0 || partition_tokens > 65536))
     return PKV_ERR_BAD_SHAPE;
   if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
   if (!std::isfinite(scale)) return PKV_ERR_BAD_SHAPE;
@@ -273,11 +298,12 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   const int D = pool.head_dim;
   const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
   CUtensorMap kmap, vmap;
+  // one box = 16 token rows of one (page, KV head): a page, or half of one
   if ((st = make_map(&kmap, k_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
-                     pool.page_size, 1, true)) != PKV_OK)
+                     pkv::decode::kBoxRows, 1, true)) != PKV_OK)
     return st;
   if ((st = make_map(&vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, D,
-                     pool.page_size, 1, false)) != PKV_OK)
+                     pkv::decode::kBoxRows, 1, false)) != PKV_OK)
     return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   pkv::decode::Params prm;
@@ -315,17 +341,12 @@ int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_
   DeviceInfo dev;
   int st;
   if ((st = current_device(&dev)) != PKV_OK) return st;
-  const long long rows = static_cast<long long>(batch) * num_q_heads;
-  const long long blocks = (rows + 3) / 4;
-  if (blocks > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if (head_dim == 128)
-    pkv::decode::combine_kernel<128><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
-        part_o, part_lse, num_splits, batch, num_q_heads, max_splits, static_cast<uint16_t*>(out), out_lse, 0);
-  else
-    pkv::decode::combine_kernel<64><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
-        part_o, part_lse, num_splits, batch, num_q_heads, max_splits, static_cast<uint16_t*>(out), out_lse, 0);
-  return launch_status();
+    return launch_combine<128>(part_o, part_lse, num_splits, batch, num_q_heads, max_splits,
+                               static_cast<uint16_t*>(out), out_lse, 0, s);
+  return launch_combine<64>(part_o, part_lse, num_splits, batch, num_q_heads, max_splits,
+                            static_cast<uint16_t*>(out), out_lse, 0, s);
 }
 
 int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch,
