@@ -205,6 +205,40 @@ PKV_API int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_le
                                    const int32_t* page_table, int32_t max_pages, float scale,
                                    void* out, pkv_stream_t stream);
 
+/*
+ * pkv_paged_attn_decode_static -- pkv_paged_attn_decode without a
+ * caller-provided workspace.  (The source pages have no counterpart: this is
+ * a deployment convenience, not part of the method.)
+ *
+ * For callers that cannot allocate device memory when they run decode --
+ * code running inside another allocator's callbacks, plugins whose host
+ * framework hands out only input and output buffers, processes that must not
+ * grow their device footprint once serving has started.  The split-K scratch
+ * lives in one array of 32 MiB compiled into the library, which every GPU
+ * that loads the library holds until the process exits.  The call allocates
+ * and frees nothing.
+ *
+ *   Arguments: as pkv_paged_attn_decode, minus workspace/workspace_bytes.
+ *   Limit: returns PKV_ERR_WORKSPACE, launching nothing, when
+ *     pkv_decode_workspace_bytes(batch, num_q_heads, head_dim,
+ *     max_pages * page_size, partition_tokens) exceeds 32 MiB.
+ *   First call per device: looks up the array's device address with
+ *     cudaGetSymbolAddress (for the device current at the time); make that
+ *     first call before any stream capture begins.
+ *   Sharing: every call on a device uses the same array, and the array keeps
+ *     the previous call's contents; each call clears the scheduling counters
+ *     at its start (an asynchronous memset on `stream`).  Calls whose work
+ *     overlaps on the GPU (other streams, other host threads) race on the
+ *     array and give wrong results: issue them one after another on one
+ *     stream.
+ */
+PKV_API int pkv_paged_attn_decode_static(const void* q, int32_t batch, int32_t num_q_heads,
+                                         const void* k_pool, const void* v_pool,
+                                         pkv_pool_desc pool, const int32_t* page_table,
+                                         int32_t max_pages, const int32_t* kv_lens, float scale,
+                                         int32_t partition_tokens, void* out, float* out_lse,
+                                         pkv_stream_t stream);
+
 /* Human-readable name of a pkv_status value (static string). */
 PKV_API const char* pkv_status_string(int status);
 

@@ -27,6 +27,7 @@ __all__ = [
     "PkvError", "LIB_PATH", "pool_desc", "pkv_kv_append", "pkv_decode_workspace_bytes",
     "pkv_paged_attn_decode", "pkv_split_k_combine", "pkv_paged_attn_chunked_prefill",
     "pkv_status_string", "pkv_device_error_flags", "decode_workspace",
+    "pkv_paged_attn_decode_static",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -220,4 +221,47 @@ def pkv_paged_attn_chunked_prefill(q, cu_q_lens, ctx_offsets, k_pool, v_pool, pa
         _ptr(q), _ptr(cu_q_lens), B, hq, total_q, int(max_q_len), _ptr(ctx_offsets),
         _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table), page_table.shape[1],
         float(scale), _ptr(out), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------ decode with built-in scratch
+_static_decode = _lib.pkv_paged_attn_decode_static
+_static_decode.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                           ctypes.c_void_p, _PoolDesc, ctypes.c_void_p, ctypes.c_int32,
+                           ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
+                           ctypes.c_void_p, ctypes.c_void_p]
+_static_decode.restype = ctypes.c_int
+
+
+def pkv_paged_attn_decode_static(q, k_pool, v_pool, page_table, kv_lens, scale,
+                                 partition_tokens=0, out=None, out_lse=None, stream=None):
+    """Decode attention like pkv_paged_attn_decode, but with the library's own
+    fixed 32 MiB scratch instead of a workspace, for callers that cannot
+    allocate device memory when they run decode (code inside another
+    allocator's callbacks, plugins that receive only their input and output
+    buffers, servers that must not grow their footprint after start-up).
+
+    Allocates nothing itself when ``out`` (and ``out_lse``, if wanted) are
+    given.  Every call on a device shares the one scratch array, so calls must
+    not overlap on the GPU; the first call on a device looks the array up and
+    should come before any stream capture.  Sizes whose split-K scratch
+    exceeds 32 MiB are rejected (PkvError, status PKV_ERR_WORKSPACE).
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    _need(page_table, "page_table", torch.int32, 2)
+    _need(kv_lens, "kv_lens", torch.int32, 1)
+    B, hq, d = q.shape
+    if page_table.shape[0] != B or kv_lens.shape[0] != B:
+        raise ValueError("page_table / kv_lens rows must equal the batch")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 3)
+    if out_lse is not None:
+        _need(out_lse, "out_lse", torch.float32, 2)
+    _check("pkv_paged_attn_decode_static", _static_decode(
+        _ptr(q), B, hq, _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table),
+        page_table.shape[1], _ptr(kv_lens), float(scale), int(partition_tokens), _ptr(out),
+        _ptr(out_lse), _stream(stream)))
     return out

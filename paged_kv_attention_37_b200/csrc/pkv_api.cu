@@ -413,3 +413,79 @@ int pkv_device_error_flags(uint32_t* flags, int clear) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Decode with built-in scratch: pkv_paged_attn_decode_static
+//
+// Some callers cannot allocate device memory at the moment they run decode:
+// code that runs inside another allocator's callbacks (where allocating would
+// re-enter it), plugins whose host framework hands out only the input and
+// output buffers and owns every other allocation, and processes that must not
+// grow their device footprint once serving has started.  This entry point
+// keeps the split-K scratch of pkv_paged_attn_decode (the per-split partials
+// and the two work-scheduling counters) in one fixed array compiled into the
+// library instead of in a caller-provided workspace, and allocates nothing.
+// ===========================================================================
+
+namespace {
+// Size of the built-in scratch.  Every GPU that loads this library holds this
+// much device memory for it until the process exits.
+constexpr size_t kStaticScratchBytes = size_t{32} << 20;  // 32 MiB
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_static_decode_scratch[kStaticScratchBytes];
+
+namespace {
+// Device address of g_static_decode_scratch, looked up once per device.  In
+// host code the array's name only stands in for the symbol; kernels must be
+// given the address the runtime reports for the current device.
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_decode_scratch) != cudaSuccess || p == nullptr)
+      return PKV_ERR_CUDA;
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return PKV_OK;
+}
+}  // namespace
+
+extern "C" int pkv_paged_attn_decode_static(const void* q, int32_t batch, int32_t num_q_heads,
+                                            const void* k_pool, const void* v_pool,
+                                            pkv_pool_desc pool, const int32_t* page_table,
+                                            int32_t max_pages, const int32_t* kv_lens, float scale,
+                                            int32_t partition_tokens, void* out, float* out_lse,
+                                            pkv_stream_t stream) {
+  // the argument checks of pkv_paged_attn_decode, so that a bad call leaves
+  // the scratch untouched
+  if (batch < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
+  int st = check_pool(pool);
+  if (st != PKV_OK) return st;
+  int group = 0;
+  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
+  const long long max_kv = static_cast<long long>(max_pages) * pool.page_size;
+  if (max_kv > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
+  if (batch > 0 && (!q || !k_pool || !v_pool || !page_table || !kv_lens || !out))
+    return PKV_ERR_NULL_POINTER;
+  if (batch > 0 && (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out)))
+    return PKV_ERR_MISALIGNED;
+  const size_t need = pkv_decode_workspace_bytes(batch, num_q_heads, pool.head_dim,
+                                                 static_cast<int32_t>(max_kv), partition_tokens);
+  if (need > kStaticScratchBytes) return PKV_ERR_WORKSPACE;  // beyond the built-in 32 MiB
+  if (batch == 0) return PKV_OK;
+  void* scratch = nullptr;
+  if ((st = static_scratch(&scratch)) != PKV_OK) return st;
+  // The array keeps whatever the previous call left; the scheduling counters
+  // at its start must be zero when the decode kernel begins.
+  if (cudaMemsetAsync(scratch, 0, 256, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PKV_ERR_CUDA;
+  return pkv_paged_attn_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages,
+                               kv_lens, scale, partition_tokens, scratch, kStaticScratchBytes, out,
+                               out_lse, stream);
+}
