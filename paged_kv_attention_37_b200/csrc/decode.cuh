@@ -40,7 +40,13 @@
 namespace pkv {
 namespace decode {
 
-constexpr int kBoxRows = 16;     // token rows per TMA box (a page, or half of one)
+constexpr int kBoxRows = 16;     // token rows per copy unit (a page, or half of one)
+#ifndef PKV_DECODE_CPASYNC
+#define PKV_DECODE_CPASYNC 1
+#endif
+// Stage fills: 16-byte cp.async copies issued by all 32 lanes (completion
+// tracked per thread with commit/wait groups), or TMA issued by lane 0.
+constexpr bool kCpAsync = PKV_DECODE_CPASYNC != 0;
 template <int D>
 struct Chunk {
   static constexpr int kLanesPerToken = D / 64;        // each lane scores 64 elements
@@ -59,6 +65,8 @@ constexpr int kLast = 2;   // last chunk of an item
 
 struct Params {
   const uint16_t* q;          // bf16 [B][Hq][D]
+  const uint16_t* k_pool;     // bf16 [num_pages][Hkv][P][D]
+  const uint16_t* v_pool;     // bf16 [num_pages][Hkv][P][D]
   const int32_t* page_table;  // [B][max_pages]
   const int32_t* kv_lens;     // [B]
   uint16_t* out;              // bf16 [B][Hq][D]
@@ -83,7 +91,8 @@ struct ItemInfo {
 template <int D, int G, int NS>
 struct Layout {
   static constexpr int kTok = Chunk<D>::kTokens;
-  static constexpr int kKBytes = kTok * D * 2;  // [D/64][kTok rows][128 B], swizzled
+  // K: [kTok rows][D/64 parts][128 B], 128-byte swizzled per 128-byte line
+  static constexpr int kKBytes = kTok * D * 2;
   static constexpr int kVBytes = kTok * D * 2;  // [kTok rows][D] bf16
   static constexpr int kStageBytes = kKBytes + kVBytes;
   // scaled query pairs, fp32 [D/64 parts][32 pairs][G][2]; each part starts
@@ -112,6 +121,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
@@ -316,7 +332,40 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
         pages[b] = __shfl_sync(0xffffffffu, pid_cur, pi & 31);
       }
     }
-    if (lane == 0) {
+    if constexpr (kCpAsync) {
+      // all lanes copy 16-byte pieces; K goes to its swizzled position
+      if (lane == 0) fifo[stage] = ChunkInfo{it_slot, ntok, flags, it_qslot};
+      if (ntok > 0) {
+        const uint32_t st = wbase + stage * LY::kStageBytes;
+#pragma unroll
+        for (int b = 0; b < Chunk<D>::kBoxes; ++b) {
+          if (b >= nbox) break;
+          int page = pages[b];
+          if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) {
+            if (lane == 0) raise_flag(PKV_FLAG_BAD_PAGE);  // read page 0: wrong values, no stray access
+            page = 0;
+          }
+          const size_t row0 = (static_cast<size_t>(page) * p.Hkv + it_g) * p.P + ((tok0 + b * kBoxRows) & (p.P - 1));
+          const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + row0 * D);
+          const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + row0 * D);
+          constexpr int kPieces = kBoxRows * D / 8;  // 16-byte pieces per 16-row box
+#pragma unroll
+          for (int i = lane; i < kPieces; i += 32) {
+            const int t = i / (D / 8), c16 = i % (D / 8);
+            const int line = (b * kBoxRows + t) * (D / 64) + (c16 >> 3);
+            cp_async16(st + line * 128 + (((c16 & 7) ^ (line & 7)) << 4), ksrc + i * 16);
+            cp_async16(st + LY::kKBytes + ((b * kBoxRows + t) * D + c16 * 8) * 2, vsrc + i * 16);
+          }
+        }
+        if (it_k == 0) {
+          const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(
+              p.q + (static_cast<size_t>(it_r) * p.Hq + static_cast<size_t>(it_g) * G) * D);
+          const uint32_t qdst = wbase + LY::kQInOff + it_qslot * (G * D * 2);
+#pragma unroll
+          for (int i = lane; i < G * D * 2 / 16; i += 32) cp_async16(qdst + i * 16, qsrc + i * 16);
+        }
+      }
+    } else if (lane == 0) {
       fifo[stage] = ChunkInfo{it_slot, ntok, flags, it_qslot};
       if (ntok > 0) {
         const bool with_q = it_k == 0;
@@ -327,15 +376,19 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
 #pragma unroll
         for (int b = 0; b < Chunk<D>::kBoxes; ++b) {
           if (b >= nbox) break;
-          if (static_cast<unsigned>(pages[b]) >= static_cast<unsigned>(p.num_pages))
-            raise_flag(PKV_FLAG_BAD_PAGE);  // TMA reads zeros out of bounds
-          const int row = pages[b] * p.Hkv + it_g;
+          int page = pages[b];
+          if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) {
+            raise_flag(PKV_FLAG_BAD_PAGE);  // read page 0 instead: wrong values, no stray access
+            page = 0;
+          }
+          const int row = page * p.Hkv + it_g;
           const int r0 = (tok0 + b * kBoxRows) & (p.P - 1);
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(st + h * (kTok * 128) + b * (kBoxRows * 128), &kmap, 64 * h, r0, row,
-                        full_bar(stage));
-          tma_load_3d(st + LY::kKBytes + b * (kBoxRows * D * 2), &vmap, 0, r0, row, full_bar(stage));
+          // K: one tensor box = 16 token rows x all D/64 parts, swizzled;
+          // V: the same 16 rows are one contiguous run of the pool
+          tma_load_4d(st + b * (kBoxRows * D * 2), &kmap, 0, 0, r0, row, full_bar(stage));
+          bulk_load(st + LY::kKBytes + b * (kBoxRows * D * 2),
+                    p.v_pool + (static_cast<size_t>(row) * p.P + r0) * D, kBoxRows * D * 2,
+                    full_bar(stage));
         }
         if (with_q)
           bulk_load(wbase + LY::kQInOff + it_qslot * (G * D * 2),
@@ -353,15 +406,25 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
   // ================================ compute side ================================
   // token of this lane, and which 64-element part of d it scores
   const int tl = kLPT == 2 ? (lane & 15) : lane, hh = kLPT == 2 ? (lane >> 4) : 0;
-  const uint32_t swz = static_cast<uint32_t>(tl & 7) << 4;
   float2 o2[G][DPL / 2];
   float m[G], l[G];
+  // Every issue attempt commits one cp.async group (possibly empty), so the
+  // group of chunk n is complete once at most NS-2 newer groups are pending.
   int issued = 0;
-  while (issued < NS - 1 && issue(issued)) ++issued;
+  for (int i = 0; i < NS - 1; ++i) {
+    const bool ok = issued == i && issue(issued);
+    if constexpr (kCpAsync) cp_async_commit();
+    if (ok) ++issued;
+  }
   int n = 0;
   for (; n < issued; ++n) {
     const int stage = n % NS;
-    if (!mbar_wait(full_bar(stage), (n / NS) & 1)) break;
+    if constexpr (kCpAsync) {
+      cp_async_wait<NS - 2>();
+      __syncwarp();
+    } else {
+      if (!mbar_wait(full_bar(stage), (n / NS) & 1)) break;
+    }
     const ChunkInfo ci = fifo[stage];
     const int ntok = ci.ntok;
     if (ci.flags & kFirst) {
@@ -387,8 +450,12 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
     }
     // keep NS-1 chunks in flight: refill the stage chunk n-1 used
     __syncwarp();
-    fence_proxy_async_smem();
-    if (issue(issued)) ++issued;
+    if constexpr (!kCpAsync) fence_proxy_async_smem();
+    {
+      const bool ok = issue(issued);
+      if constexpr (kCpAsync) cp_async_commit();
+      if (ok) ++issued;
+    }
 
     if (ntok > 0) {
       const uint8_t* stp = wb + stage * LY::kStageBytes;
@@ -396,7 +463,11 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
       float2 acc[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
-      const uint8_t* krow = stp + hh * (kTok * 128) + tl * 128;
+      // this lane's 128-byte line of K: token tl, part hh; its swizzle phase
+      // is the line index mod 8
+      const int kline = tl * (D / 64) + hh;
+      const uint8_t* krow = stp + kline * 128;
+      const uint32_t swz = static_cast<uint32_t>(kline & 7) << 4;
       const uint8_t* qh = reinterpret_cast<const uint8_t*>(qf) + hh * LY::kQHalfBytes;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {

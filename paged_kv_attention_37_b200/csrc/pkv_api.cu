@@ -55,6 +55,23 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// 4-D bf16 tensor map over a pool, viewing each token row as D/64 parts of
+// 64 elements: dims (64, D/64, P, pages*Hkv), 128-byte swizzle.
+int make_pool_map_parts(CUtensorMap* map, const void* base, const pkv_pool_desc& pool, uint32_t rows_box) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return PKV_ERR_TENSOR_MAP;
+  const uint64_t D = pool.head_dim;
+  const cuuint64_t dims[4] = {64, D / 64, static_cast<cuuint64_t>(pool.page_size),
+                              static_cast<cuuint64_t>(pool.num_pages) * pool.num_kv_heads};
+  const cuuint64_t strides[3] = {128, D * 2, static_cast<cuuint64_t>(pool.page_size) * D * 2};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(D / 64), rows_box, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_TENSOR_MAP;
+}
+
 // 3-D bf16 tensor map: dims[0] innermost (elements), strides in bytes of
 // dims 1 and 2.
 int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
@@ -299,15 +316,15 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
   CUtensorMap kmap, vmap;
   // one box = 16 token rows of one (page, KV head): a page, or half of one
-  if ((st = make_map(&kmap, k_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
-                     pkv::decode::kBoxRows, 1, true)) != PKV_OK)
-    return st;
+  if ((st = make_pool_map_parts(&kmap, k_pool, pool, pkv::decode::kBoxRows)) != PKV_OK) return st;
   if ((st = make_map(&vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, D,
                      pkv::decode::kBoxRows, 1, false)) != PKV_OK)
     return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   pkv::decode::Params prm;
   prm.q = static_cast<const uint16_t*>(q);
+  prm.k_pool = static_cast<const uint16_t*>(k_pool);
+  prm.v_pool = static_cast<const uint16_t*>(v_pool);
   prm.page_table = page_table;
   prm.kv_lens = kv_lens;
   prm.out = static_cast<uint16_t*>(out);
