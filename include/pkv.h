@@ -97,7 +97,8 @@ enum pkv_status {
 #define PKV_FLAG_BAD_LENGTH     0x2u  /* a kv_len/ctx/chunk length < 0 or beyond max_pages*page_size */
 #define PKV_FLAG_BAD_SLOT       0x4u  /* kv_append slot >= num_pages*page_size (row skipped) */
 #define PKV_FLAG_BAD_QUERY_ROWS 0x8u  /* cu_q_lens not non-decreasing within [0, total_q] */
-#define PKV_FLAG_BAD_PAGE       0x10u /* a page-table entry outside [0, num_pages) was read (as zeros) */
+#define PKV_FLAG_BAD_PAGE       0x10u /* a page-table entry outside [0, num_pages) was seen (page 0 or zeros read instead) */
+#define PKV_FLAG_INTERNAL       0x20u /* a kernel found an internal invariant broken and skipped its work */
 
 /*
  * pkv_kv_append -- write the K/V rows of this step's new tokens into pool

@@ -37,6 +37,7 @@ FLAG_BAD_LENGTH = 0x2
 FLAG_BAD_SLOT = 0x4
 FLAG_BAD_QUERY_ROWS = 0x8
 FLAG_BAD_PAGE = 0x10
+FLAG_INTERNAL = 0x20
 
 
 class PkvError(RuntimeError):

@@ -199,13 +199,19 @@ int dispatch_decode_group(int group, const pkv::decode::Params& prm, const CUten
 }
 
 // ----------------------------------------------------------- prefill launch
+#ifndef PKV_PREFILL_BN
+#define PKV_PREFILL_BN 64
+#endif
+
 template <int D, int G>
 int launch_prefill(const pkv::prefill::Params& prm, const CUtensorMap& qmap, const CUtensorMap& kmap,
                    const CUtensorMap& vmap, int32_t max_q_len, cudaStream_t stream) {
-  using LY = pkv::prefill::Layout<D>;
-  auto kernel = pkv::prefill::prefill_kernel<D, G>;
-  // at least ~116 KB so that one CTA (and its 512 TMEM columns) owns an SM
-  const size_t smem = std::max<size_t>(LY::kBytes, 116 * 1024);
+  constexpr int BN = PKV_PREFILL_BN;  // keys per tile
+  using LY = pkv::prefill::Layout<D, BN>;
+  auto kernel = pkv::prefill::prefill_kernel<D, G, BN>;
+  // BN=64: about half an SM's shared memory, so two CTAs (with 256 TMEM
+  // columns each) share an SM; BN=128: one CTA and 512 columns per SM
+  const size_t smem = BN == 64 ? LY::kBytes : std::max<size_t>(LY::kBytes, 116 * 1024);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return PKV_ERR_CUDA;
@@ -214,7 +220,9 @@ int launch_prefill(const pkv::prefill::Params& prm, const CUtensorMap& qmap, con
   const long long blocks = tiles * prm.Hkv * prm.B;
   if (blocks == 0) return PKV_OK;
   if (blocks > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
-  kernel<<<static_cast<unsigned>(blocks), pkv::prefill::kThreads, smem, stream>>>(qmap, kmap, vmap, prm);
+  pkv::prefill::Params args = prm;
+  args.qtiles = static_cast<int32_t>(tiles);
+  kernel<<<static_cast<unsigned>(blocks), pkv::prefill::kThreads, smem, stream>>>(qmap, kmap, vmap, args);
   return launch_status();
 }
 
@@ -376,7 +384,7 @@ int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int3
   if (st != PKV_OK) return st;
   int group = 0;
   if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
-  if (!std::isfinite(scale)) return PKV_ERR_BAD_SHAPE;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return PKV_ERR_BAD_SHAPE;
   if (batch == 0 || total_q == 0 || max_q_len == 0) return PKV_OK;
   if (!q || !cu_q_lens || !ctx_offsets || !k_pool || !v_pool || !page_table || !out)
     return PKV_ERR_NULL_POINTER;

@@ -9,13 +9,15 @@
 //
 // Tile: one CTA computes 128 query rows = 128/G consecutive chunk positions
 // x the G query heads of one KV head (GQA packing: each K/V tile in shared
-// memory serves all G heads).  Keys stream in tiles of 128 (8 pages of 16, or
-// 4 of 32), gathered page by page with TMA into 128-byte-swizzled tiles.
-//   S = Q K^T   : M=128, N=128, K=d  -> TMEM (two buffers, double-buffered)
+// memory serves all G heads).  Keys stream in tiles of BN (64: 4 pages of 16
+// or 2 of 32), gathered page by page with TMA into 128-byte-swizzled tiles.
+//   S = Q K^T   : M=128, N=BN, K=d  -> TMEM (two buffers, double-buffered)
 //   softmax     : one thread per TMEM lane (= one query row), log2 domain,
 //                 lazy rescale of O only when the running max grows by > 2^8
-//   O += P V    : M=128, N=d, K=128; P (bf16) staged in shared memory,
+//   O += P V    : M=128, N=d, K=BN; P (bf16) staged in shared memory,
 //                 V used as an MN-major operand straight from its tile
+// With BN=64 a CTA needs ~112 KB of shared memory and 256 TMEM columns, so
+// two CTAs share an SM and one CTA's softmax overlaps the other's MMAs.
 // Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer (one
 // thread), warps 2..5 softmax and epilogue.
 #pragma once
@@ -26,10 +28,7 @@ namespace pkv {
 namespace prefill {
 
 constexpr int kM = 128;  // query rows per CTA
-constexpr int kN = 128;  // keys per tile
 constexpr int kThreads = 192;
-constexpr int kTmemCols = 512;
-constexpr int kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 256x
 
 struct Params {
@@ -38,41 +37,63 @@ struct Params {
   const int32_t* page_table;   // [B][max_pages]
   uint16_t* out;               // bf16 [total_q][Hq][D]
   int32_t B, Hq, Hkv, P, max_pages, num_pages, total_q;
+  int32_t qtiles;  // query tiles per request in the grid (ceil(max_q_len / rows per tile))
   float scale_log2;
 };
 
-template <int D>
+#ifndef PKV_PREFILL_ORDER
+#define PKV_PREFILL_ORDER 1
+#endif
+
+template <int D, int BN>
 struct Layout {
-  static constexpr int kHalf = kM * 128;            // one 64-column half of a 128-row tile
-  static constexpr int kQOff = 0;                   // [D/64][128 rows][128 B]
-  static constexpr int kTileBytes = (D / 64) * kHalf;
-  static constexpr int kKOff = kQOff + kTileBytes;  // 2 stages
-  static constexpr int kVOff = kKOff + 2 * kTileBytes;
-  static constexpr int kPOff = kVOff + 2 * kTileBytes;  // [2 halves][128 rows][128 B]
-  static constexpr int kBarOff = kPOff + 2 * kHalf;
-  // barriers: q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull, pvdone, final
-  static constexpr int kNumBars = 14;
+  static constexpr int kQHalf = kM * 128;               // one 64-column half of the Q or P tile
+  static constexpr int kKVHalf = BN * 128;              // one 64-column half of a K or V tile
+  static constexpr int kQOff = 0;                       // [D/64][128 rows][128 B]
+  static constexpr int kKVTile = (D / 64) * kKVHalf;    // [D/64][BN rows][128 B]
+  static constexpr int kKOff = kQOff + (D / 64) * kQHalf;  // 2 stages
+  static constexpr int kVOff = kKOff + 2 * kKVTile;
+  static constexpr int kPOff = kVOff + 2 * kKVTile;     // [BN/64][128 rows][128 B]
+  static constexpr int kBarOff = kPOff + (BN / 64) * kQHalf;
+  static constexpr int kTmemCols = 2 * BN + D <= 256 ? 256 : 512;  // S0, S1, O
+  static constexpr int kColS0 = 0, kColS1 = BN, kColO = 2 * BN;
+  // barriers: q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull, pvdone, final, sfree[2]
+  static constexpr int kNumBars = 16;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
-  static constexpr size_t kBytes = kTmemSlotOff + 16 + 1024;
+  static constexpr size_t kBytes = kTmemSlotOff + 16;  // the base is 1024-byte aligned
 };
 
 enum Bar { kQ = 0, kKFull = 1, kKEmpty = 3, kVFull = 5, kVEmpty = 7, kSFull = 9, kPFull = 11,
-           kPVDone = 12, kFinal = 13 };
+           kPVDone = 12, kFinal = 13, kSFree = 14 };
 
-template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int G, int BN>
+__global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const Params p) {
-  using LY = Layout<D>;
+  using LY = Layout<D, BN>;
+  constexpr int kN = BN;        // keys per tile
+  constexpr int kTmemCols = LY::kTmemCols;
+  constexpr int kColS0 = LY::kColS0, kColS1 = LY::kColS1, kColO = LY::kColO;
   constexpr int QPOS = kM / G;  // chunk positions per tile
   constexpr uint32_t kIdescS = idesc_bf16_f32(kM, kN, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, D, false, true);
 
-  // ---- which tile: heaviest (last) q-tiles of every request first
-  const int r = blockIdx.x % p.B;
-  const int rest = blockIdx.x / p.B;
-  const int g = rest % p.Hkv;
-  const int qt_rev = rest / p.Hkv;
+  // ---- which tile.  Order 1: the query tiles of one (request, KV head) are
+  // adjacent, heaviest (last) first, so the CTAs that read the same keys run
+  // together and share them through L2.  Order 0: heaviest tiles of every
+  // request first.
+  int r, g, qt_rev;
+  if (PKV_PREFILL_ORDER == 1) {
+    qt_rev = blockIdx.x % p.qtiles;
+    const int rest = blockIdx.x / p.qtiles;
+    g = rest % p.Hkv;
+    r = rest / p.Hkv;
+  } else {
+    r = blockIdx.x % p.B;
+    const int rest = blockIdx.x / p.B;
+    g = rest % p.Hkv;
+    qt_rev = rest / p.Hkv;
+  }
   const int q0 = p.cu_q_lens[r], q1 = p.cu_q_lens[r + 1];
   const int n_r = q1 - q0;
   if (q0 < 0 || n_r < 0 || q1 > p.total_q) {
@@ -92,10 +113,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kv_end = pos_lo + rows_valid;                // keys 0 .. kv_end-1 are used
   const int nt = (kv_end + kN - 1) / kN;                 // key tiles
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 128-byte swizzle atoms need 1024-byte alignment; the declaration asks
+  // for it, and a misaligned base (never expected) is refused, not used
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_addr(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) raise_flag(PKV_FLAG_INTERNAL);
+    return;
+  }
   auto bar = [&](int i) { return sbase + LY::kBarOff + 8u * i; };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + LY::kTmemSlotOff);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -108,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kVFull + i), 1);
       mbar_init(bar(kVEmpty + i), 1);
       mbar_init(bar(kSFull + i), 1);
+      mbar_init(bar(kSFree + i), 128);
     }
     mbar_init(bar(kPFull), 128);
     mbar_init(bar(kPVDone), 1);
@@ -121,8 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   const uint32_t sQ = sbase + LY::kQOff;
-  auto sK = [&](int b) { return sbase + LY::kKOff + b * LY::kTileBytes; };
-  auto sV = [&](int b) { return sbase + LY::kVOff + b * LY::kTileBytes; };
+  auto sK = [&](int b) { return sbase + LY::kKOff + b * LY::kKVTile; };
+  auto sV = [&](int b) { return sbase + LY::kVOff + b * LY::kKVTile; };
   const uint32_t sP = sbase + LY::kPOff;
 
   if (warp == 0) {
@@ -135,87 +162,130 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(bar(kQ), kM * D * 2);
 #pragma unroll
       for (int h = 0; h < D / 64; ++h)
-        tma_load_3d(sQ + h * LY::kHalf, &qmap, 64 * h, g * G, q0 + qt * QPOS, bar(kQ));
+        tma_load_3d(sQ + h * LY::kQHalf, &qmap, 64 * h, g * G, q0 + qt * QPOS, bar(kQ));
     }
-    bool ok = true;
-    for (int j = 0; j < nt && ok; ++j) {
+    // K of tile j only waits for its stage (freed when S of tile j-2 is
+    // done); V trails one tile behind, since P.V of a tile runs after its
+    // softmax.  Coupling the two would make every S wait for an earlier P.V.
+    // page ids of tile j: the request's page-table entries are read 32 at a
+    // time, the next 32 already in flight, so no TMA issue waits on them
+    const int total_pages = (kv_end + p.P - 1) / p.P;
+    int pid_base = 0;
+    int pid_cur = lane < total_pages ? __ldg(ptab + lane) : -1;
+    int pid_next = 32 + lane < total_pages ? __ldg(ptab + 32 + lane) : -1;
+    auto tile_pages = [&](int j) {
+      const int first = j * kN / p.P;
+      const int npg = (min(kN, kv_end - j * kN) + p.P - 1) / p.P;
+      while (first >= pid_base + 32) {
+        pid_base += 32;
+        pid_cur = pid_next;
+        pid_next = pid_base + 32 + lane < total_pages ? __ldg(ptab + pid_base + 32 + lane) : -1;
+      }
+      // a tile's pages never straddle a 32-entry window: kN/P divides 32
+      const int src = (first - pid_base) + (lane < npg ? lane : 0);
+      const int pid = __shfl_sync(0xffffffffu, pid_cur, src & 31);
+      return make_int2(npg, lane < npg ? pid : -1);
+    };
+    auto issue_tile = [&](int j, int2 pg, int which) {  // which: 0 = K, 1 = V
       const int b = j & 1;
-      const int key0 = j * kN;
-      const int nkeys = min(kN, kv_end - key0);
-      const int npg = (nkeys + p.P - 1) / p.P;
-      const int pid = lane < npg ? __ldg(ptab + key0 / p.P + lane) : -1;
-      if (j >= 2) {
-        ok = mbar_wait(bar(kKEmpty + b), ((j >> 1) - 1) & 1);
-        if (ok) ok = mbar_wait(bar(kVEmpty + b), ((j >> 1) - 1) & 1);
-        if (!ok) break;
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(kKFull + b), static_cast<uint32_t>(npg * p.P * D * 2));
-      }
-      for (int pi = 0; pi < npg; ++pi) {
-        const int page = __shfl_sync(0xffffffffu, pid, pi);
+      const uint32_t full = bar((which ? kVFull : kKFull) + b);
+      const CUtensorMap* map = which ? &vmap : &kmap;
+      const uint32_t dst = which ? sV(b) : sK(b);
+      if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(pg.x * p.P * D * 2));
+      for (int pi = 0; pi < pg.x; ++pi) {
+        const int page = __shfl_sync(0xffffffffu, pg.y, pi);
         if (lane == 0) {
-          if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) raise_flag(PKV_FLAG_BAD_PAGE);
+          if (which == 0 && static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages))
+            raise_flag(PKV_FLAG_BAD_PAGE);  // TMA reads zeros out of bounds
           const int row = page * p.Hkv + g;
 #pragma unroll
           for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(sK(b) + h * LY::kHalf + pi * p.P * 128, &kmap, 64 * h, 0, row, bar(kKFull + b));
+            tma_load_3d(dst + h * LY::kKVHalf + pi * p.P * 128, map, 64 * h, 0, row, full);
         }
       }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(kVFull + b), static_cast<uint32_t>(npg * p.P * D * 2));
+    };
+    bool ok = true;
+    int2 pg_prev = make_int2(0, -1);
+    for (int j = 0; j <= nt && ok; ++j) {
+      int2 pg = make_int2(0, -1);
+      if (j < nt) {
+        pg = tile_pages(j);
+        if (j >= 2 && !(ok = mbar_wait(bar(kKEmpty + (j & 1)), ((j >> 1) - 1) & 1))) break;
+        issue_tile(j, pg, 0);
       }
-      for (int pi = 0; pi < npg; ++pi) {
-        const int page = __shfl_sync(0xffffffffu, pid, pi);
-        if (lane == 0) {
-          const int row = page * p.Hkv + g;
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(sV(b) + h * LY::kHalf + pi * p.P * 128, &vmap, 64 * h, 0, row, bar(kVFull + b));
-        }
+      if (j >= 1) {
+        const int jv = j - 1;
+        if (jv >= 2 && !(ok = mbar_wait(bar(kVEmpty + (jv & 1)), ((jv >> 1) - 1) & 1))) break;
+        issue_tile(jv, pg_prev, 1);
       }
+      pg_prev = pg;
       __syncwarp();
     }
   } else if (warp == 1) {
     // ============================ MMA issuer =============================
+    // Two streams of MMAs: S of tile j (needs K(j) and a free S buffer) and
+    // P.V of tile j (needs P(j) and V(j)).  The issuer takes whichever is
+    // ready, P.V first, so a late K tile never holds up a P.V the softmax
+    // warps are waiting for.  S of tile j+2 reuses the buffer of tile j as
+    // soon as the softmax warps have read S(j).
     bool ok = mbar_wait(bar(kQ), 0);
-    auto issue_pv = [&](int i) -> bool {
+    auto do_pv = [&](int i) {
       const int b = i & 1;
-      if (!mbar_wait(bar(kPFull), i & 1)) return false;
-      if (!mbar_wait(bar(kVFull + b), (i >> 1) & 1)) return false;
       tc_fence_after_sync();
       if (lane == 0) {
 #pragma unroll
         for (int ks = 0; ks < kN / 16; ++ks) {
-          const uint64_t a = smem_desc_sw128(sP + (ks >> 2) * LY::kHalf + (ks & 3) * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(sV(b) + ks * 16 * 128, LY::kHalf, 1024);
+          const uint64_t a = smem_desc_sw128(sP + (ks >> 2) * LY::kQHalf + (ks & 3) * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(sV(b) + ks * 16 * 128, LY::kKVHalf, 1024);
           tc_mma_ss(tmem + kColO, a, bdesc, kIdescPV, i > 0 || ks > 0);
         }
         tc_commit(bar(kPVDone));
         tc_commit(bar(kVEmpty + b));
       }
       __syncwarp();
-      return true;
     };
-    for (int j = 0; j < nt && ok; ++j) {
+    auto do_s = [&](int j) {
       const int b = j & 1;
-      ok = mbar_wait(bar(kKFull + b), (j >> 1) & 1);
-      if (!ok) break;
       tc_fence_after_sync();
       if (lane == 0) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t a = smem_desc_sw128(sQ + (ks >> 2) * LY::kHalf + (ks & 3) * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(sK(b) + (ks >> 2) * LY::kHalf + (ks & 3) * 32, 16, 1024);
+          const uint64_t a = smem_desc_sw128(sQ + (ks >> 2) * LY::kQHalf + (ks & 3) * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(sK(b) + (ks >> 2) * LY::kKVHalf + (ks & 3) * 32, 16, 1024);
           tc_mma_ss(tmem + (b ? kColS1 : kColS0), a, bdesc, kIdescS, ks > 0);
         }
         tc_commit(bar(kSFull + b));
         tc_commit(bar(kKEmpty + b));
       }
       __syncwarp();
-      if (j >= 1) ok = issue_pv(j - 1);
+    };
+    for (int j = 0; j < 2 && j < nt && ok; ++j) {
+      ok = mbar_wait(bar(kKFull + (j & 1)), (j >> 1) & 1);
+      if (ok) do_s(j);
     }
-    if (ok && nt >= 1) ok = issue_pv(nt - 1);
+    int ns = 2, npv = 0;
+    uint64_t t_idle = global_timer_ns();
+    while (ok && npv < nt) {
+      int act = 0;  // 1: P.V(npv), 2: S(ns); decided by lane 0 for the whole warp
+      if (lane == 0) {
+        if (mbar_try_wait(bar(kPFull), npv & 1) && mbar_try_wait(bar(kVFull + (npv & 1)), (npv >> 1) & 1))
+          act = 1;
+        else if (ns < nt && mbar_try_wait(bar(kSFree + (ns & 1)), ((ns - 2) >> 1) & 1) &&
+                 mbar_try_wait(bar(kKFull + (ns & 1)), (ns >> 1) & 1))
+          act = 2;
+      }
+      act = __shfl_sync(0xffffffffu, act, 0);
+      if (act == 1) {
+        do_pv(npv++);
+        t_idle = global_timer_ns();
+      } else if (act == 2) {
+        do_s(ns++);
+        t_idle = global_timer_ns();
+      } else if (global_timer_ns() - t_idle > kWaitLimitNs) {
+        if (lane == 0) raise_flag(PKV_FLAG_WAIT_TIMEOUT);
+        ok = false;
+      }
+    }
     if (lane == 0) tc_commit(bar(kFinal));
     __syncwarp();
   } else {
@@ -233,16 +303,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = j & 1;
       if (!mbar_wait(bar(kSFull + b), (j >> 1) & 1)) { ok = false; break; }
       tc_fence_after_sync();
+      // raw scores of this row; hidden keys -> -inf (scale > 0, so the max
+      // of raw scores gives the max of scaled ones)
       float s[kN];
       {
         uint32_t v[kN / 32][32];
 #pragma unroll
         for (int cc = 0; cc < kN / 32; ++cc) tmem_ld_32x32b_x32(trow + (b ? kColS1 : kColS0) + cc * 32, v[cc]);
         tmem_wait_ld();
+        tc_fence_before_sync();
+        mbar_arrive(bar(kSFree + b));  // this S buffer may take the next-but-one tile
 #pragma unroll
         for (int cc = 0; cc < kN / 32; ++cc)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(v[cc][e]) * sl2;
+          for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(v[cc][e]);
       }
       const int key0 = j * kN;
       if (key0 + kN - 1 > pos_lo || key0 + kN > kv_end) {  // diagonal or ragged tile
@@ -255,22 +329,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       float mx = -INFINITY;
 #pragma unroll
       for (int e = 0; e < kN; ++e) mx = fmaxf(mx, s[e]);
-      const float mc = fmaxf(m, mx);
+      const float mc = fmaxf(m, mx * sl2);
       const bool need = mc > m + kRescaleThreshold;
       float alpha = 1.f;
       if (need) {
         alpha = fast_exp2(m - mc);
         m = mc;
       }
+      // p = 2^(s*scale*log2e - m): one FMA and one exp2 per element
       uint32_t pk[kN / 2];
-      float rowsum = 0.f;
+      float2 rs = make_float2(0.f, 0.f);
 #pragma unroll
       for (int e = 0; e < kN; e += 2) {
-        const float a0 = fast_exp2(s[e] - m), a1 = fast_exp2(s[e + 1] - m);
-        rowsum += a0 + a1;
+        const float a0 = fast_exp2(fmaf(s[e], sl2, -m)), a1 = fast_exp2(fmaf(s[e + 1], sl2, -m));
+        rs = __fadd2_rn(rs, make_float2(a0, a1));
         pk[e / 2] = pack_bf16x2(a0, a1);
       }
-      l = fmaf(l, alpha, rowsum);
+      l = fmaf(l, alpha, rs.x + rs.y);
       if (j >= 1) {
         // PV of the previous tile must be done: P is single-buffered and O
         // may need rescaling.
@@ -294,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int ch = 0; ch < kN / 8; ++ch) {
         const int half = ch >> 3, c16 = ch & 7;
-        *reinterpret_cast<uint4*>(prow + half * LY::kHalf + ((c16 ^ (row & 7)) << 4)) =
+        *reinterpret_cast<uint4*>(prow + half * LY::kQHalf + ((c16 ^ (row & 7)) << 4)) =
             make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
       }
       if (key0 + kN > kv_end) {
@@ -304,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int first = kv_end - key0;
         const int nbytes = (kN - first) * 128;
         for (int h = 0; h < D / 64; ++h) {
-          uint8_t* vz = smem + LY::kVOff + b * LY::kTileBytes + h * LY::kHalf + first * 128;
+          uint8_t* vz = smem + LY::kVOff + b * LY::kKVTile + h * LY::kKVHalf + first * 128;
           for (int off = (row) * 16; off < nbytes; off += kM * 16)
             *reinterpret_cast<uint4*>(vz + off) = make_uint4(0, 0, 0, 0);
         }

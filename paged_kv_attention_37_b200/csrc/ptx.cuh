@@ -51,18 +51,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-// Test for completion of the phase with the given parity; while it is not
-// complete the thread may be suspended in hardware for up to suspend_ns
-// before the call returns false (it does not spin).
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity,
-                                              uint32_t suspend_ns = 1000000u) {
+// Test for completion of the phase with the given parity (the hardware may
+// briefly suspend the thread before reporting "not yet").
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
