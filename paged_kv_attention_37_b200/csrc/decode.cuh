@@ -19,20 +19,25 @@
 // Every warp is independent: it takes an item, walks its page-table entries
 // (32 per warp-wide load), and keeps NS-1 chunks in flight in its own ring of
 // NS shared-memory stages of 8 KB: a chunk is 2048/d tokens (16 at d=128, 32
-// at d=64), fetched as TMA tensor boxes of 16 token rows -- K 128-byte
-// swizzled, V plain -- each box one page or half of a 32-token page,
-// completing on the stage's mbarrier, issued by lane 0 ahead of the chunk
-// being computed.  There is no cross-warp synchronisation after the planning
-// step, and the small per-warp footprint keeps 10-12 warps resident per SM.
+// at d=64), K rows then V rows, each 16-row piece one page or half of a
+// 32-token page and contiguous in the pool.  Stages are filled with 16-byte
+// cp.async copies from all lanes (or bulk copies issued by one lane).  There
+// is no cross-warp synchronisation after the planning step.
 //
-// Inside a chunk every lane scores 64 elements of one token: at d=128 lanes
-// t and t+16 share token t (one half of d each, one shuffle adds them), at
-// d=64 lane t owns token t.  Scores use q as broadcast fp32 pairs from
-// shared memory (the halves padded onto different banks), k read from the
-// swizzled block without bank conflicts, and packed fp32x2 FMAs.  The online softmax keeps a warp-uniform
-// running max and per-lane partial sums.  For P.V lane l owns output columns
-// [l*D/32, (l+1)*D/32) of every head.  At the item's end the warp writes
-// bf16 output (single-split request) or an fp32 partial and its lse.
+// Lane layout: T = d/8 lanes share one token, each holding 8 consecutive
+// elements of d, so a warp covers 32/T tokens per step.  The query rows live
+// in registers (fp32, times scale*log2(e)): lane i of a token group keeps
+// elements [8i, 8i+8) of all G heads.  A score is a dot product over the T
+// lanes of a group: a butterfly reduce-scatter over the group leaves each
+// lane with the full score of one head (G partial sums in, one out, no value
+// sent twice).  K and V are each read from shared memory exactly once, with
+// 16-byte loads that cover 512 contiguous bytes per warp (no bank
+// conflicts).  The exponentials go through a small per-warp buffer so that
+// every lane can weight its V elements for all G heads; each lane then
+// accumulates O for its 8 elements x G heads over its tokens, and the token
+// groups are summed with shuffles when the item ends.  The online softmax
+// keeps a warp-uniform running max per head that only moves when a score
+// exceeds it by more than 2^8 (in practice on an item's first chunk).
 #pragma once
 
 #include "ptx.cuh"
@@ -45,13 +50,16 @@ constexpr int kBoxRows = 16;     // token rows per copy unit (a page, or half of
 #define PKV_DECODE_CPASYNC 1
 #endif
 // Stage fills: 16-byte cp.async copies issued by all 32 lanes (completion
-// tracked per thread with commit/wait groups), or TMA issued by lane 0.
+// tracked per thread with commit/wait groups), or bulk copies issued by lane
+// 0 that complete on the stage's mbarrier.
 constexpr bool kCpAsync = PKV_DECODE_CPASYNC != 0;
 template <int D>
 struct Chunk {
-  static constexpr int kLanesPerToken = D / 64;        // each lane scores 64 elements
-  static constexpr int kTokens = 32 / kLanesPerToken;  // tokens per pipeline stage
-  static constexpr int kBoxes = kTokens / kBoxRows;    // TMA boxes per stage (per K half)
+  static constexpr int kTokens = 2048 / D;             // tokens per pipeline stage (8 KB of K+V)
+  static constexpr int kBoxes = kTokens / kBoxRows;    // 16-row pieces per stage (per K or V)
+  static constexpr int kLanesPerToken = D / 8;         // T: each lane holds 8 elements
+  static constexpr int kTokensPerStep = 32 / kLanesPerToken;
+  static constexpr int kSteps = kTokens / kTokensPerStep;
 };
 constexpr int kItemSlots = 8;    // per-warp ring of item descriptors
 constexpr int kMinAutoPartition = 256;
@@ -91,24 +99,18 @@ struct ItemInfo {
 template <int D, int G, int NS>
 struct Layout {
   static constexpr int kTok = Chunk<D>::kTokens;
-  // K: [kTok rows][D/64 parts][128 B], 128-byte swizzled per 128-byte line
-  static constexpr int kKBytes = kTok * D * 2;
-  static constexpr int kVBytes = kTok * D * 2;  // [kTok rows][D] bf16
+  static constexpr int kKBytes = kTok * D * 2;   // K rows [kTok][D] bf16
+  static constexpr int kVBytes = kTok * D * 2;   // V rows [kTok][D] bf16
   static constexpr int kStageBytes = kKBytes + kVBytes;
-  // scaled query pairs, fp32 [D/64 parts][32 pairs][G][2]; each part starts
-  // 16 bytes past a 128-byte multiple so the half-warps' broadcast reads land
-  // on different banks
-  static constexpr int kQHalfBytes = 32 * G * 8 + 16;
   static constexpr int kQInOff = NS * kStageBytes;              // bf16 [NS][G][D] staged queries
-  static constexpr int kQfOff = kQInOff + NS * G * D * 2;
-  static constexpr int kPbOff = kQfOff + (D / 64) * kQHalfBytes;  // fp32 [kTok][G][2] (p, p) pairs
+  static constexpr int kPbOff = kQInOff + NS * G * D * 2;       // fp32 [kTok][G][2] (p, p) pairs
   static constexpr int kBarOff = kPbOff + kTok * G * 8;         // NS mbarriers
   static constexpr int kFifoOff = kBarOff + NS * 8;             // NS ChunkInfo
   static constexpr int kItemOff = kFifoOff + NS * 16;           // kItemSlots ItemInfo
-  static constexpr int kWarpBytes = (kItemOff + kItemSlots * 16 + 1023) / 1024 * 1024;
+  static constexpr int kWarpBytes = (kItemOff + kItemSlots * 16 + 127) / 128 * 128;
   // after the W warp blocks: misc[4], lens[B], prefF[B+1], prefR[B+1]
   static size_t plan_bytes(int B) { return 16 + (3 * static_cast<size_t>(B) + 2) * 4; }
-  static size_t bytes(int W, int B) { return static_cast<size_t>(W) * kWarpBytes + plan_bytes(B) + 1024; }
+  static size_t bytes(int W, int B) { return static_cast<size_t>(W) * kWarpBytes + plan_bytes(B) + 128; }
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -148,21 +150,46 @@ __device__ __forceinline__ int upper_index(const int32_t* pref, int n, int x) {
   return lo;
 }
 
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x >> 1); }
+
+// Butterfly reduce-scatter of G per-head partial sums over the T lanes of a
+// token group (T a power of two, lanes [T*k, T*k+T)), then an all-reduce
+// over the group bits left over.  On return v[0] holds the full sum of head
+// (lane & (T-1)) >> (log2 T - log2 G) in every lane.
+template <int G, int T>
+__device__ __forceinline__ float reduce_scatter_heads(float (&v)[G], int lane) {
+  constexpr int LG = ilog2(G), LT = ilog2(T);
+  static_assert(LG <= LT, "more heads than lanes per token");
+#pragma unroll
+  for (int lv = 0; lv < LG; ++lv) {
+    const int off = T >> (lv + 1);   // partner distance
+    const int half = G >> (lv + 1);  // values kept after this level
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float send = upper ? v[k] : v[k + half];
+      const float keep = upper ? v[k + half] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+#pragma unroll
+  for (int off = T >> (LG + 1); off > 0; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+  return v[0];
+}
+
 template <int D, int G, int NS, int MAXW>
-__global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                                 const __grid_constant__ CUtensorMap vmap,
-                                                                 const Params p) {
+__global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p) {
   using LY = Layout<D, G, NS>;
-  constexpr int kTok = Chunk<D>::kTokens, kLPT = Chunk<D>::kLanesPerToken;
+  using CK = Chunk<D>;
+  constexpr int kTok = CK::kTokens;
+  constexpr int T = CK::kLanesPerToken, TPS = CK::kTokensPerStep, STEPS = CK::kSteps;
+  constexpr int LG = ilog2(G), LT = ilog2(T);
   const int W = blockDim.x >> 5;
   const int log2P = 31 - __clz(p.P);  // P is a power of two
-  constexpr int DPL = D / 32;  // P.V output columns per lane
-  static_assert(DPL == 2 || DPL == 4, "head_dim 64 or 128");
+  static_assert(T == 8 || T == 16, "head_dim 64 or 128");
   static_assert(NS >= 2, "at least two stages per warp");
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t* misc = reinterpret_cast<int32_t*>(smem + W * LY::kWarpBytes);
   int32_t* lens = misc + 4;
@@ -174,16 +201,13 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
   auto full_bar = [&](int i) { return wbase + LY::kBarOff + 8u * i; };
   ChunkInfo* fifo = reinterpret_cast<ChunkInfo*>(wb + LY::kFifoOff);
   ItemInfo* items = reinterpret_cast<ItemInfo*>(wb + LY::kItemOff);
-  float* qf = reinterpret_cast<float*>(wb + LY::kQfOff);
   float* pb = reinterpret_cast<float*>(wb + LY::kPbOff);
 
-  if (lane == 0) {
-    for (int i = 0; i < NS; ++i) mbar_init(full_bar(i), 1);
-    fence_barrier_init();
-  }
-  if (threadIdx.x == 0) {
-    prefetch_tensormap(&kmap);
-    prefetch_tensormap(&vmap);
+  if constexpr (!kCpAsync) {
+    if (lane == 0) {
+      for (int i = 0; i < NS; ++i) mbar_init(full_bar(i), 1);
+      fence_barrier_init();
+    }
   }
 
   // ---- plan (warp 0): clamp lengths, pick the partition, count the items:
@@ -316,12 +340,13 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
     const int ntok = it_nch == 0 ? 0 : min(kTok, it_ntok - tok0);
     const int flags = (it_k == 0 ? kFirst : 0) | (it_k + 1 >= it_nch ? kLast : 0);
     const int nbox = (ntok + kBoxRows - 1) / kBoxRows;
-    // each 16-row box lies inside one page: page-table entry (tok >> log2P),
-    // first row (tok & (P-1))
-    int pages[Chunk<D>::kBoxes];
+    // each 16-row piece lies inside one page: page-table entry (tok >> log2P),
+    // first row (tok & (P-1)); out-of-range page ids read page 0 instead
+    // (wrong values, no stray access) and raise PKV_FLAG_BAD_PAGE
+    size_t rows[CK::kBoxes];
 #pragma unroll
-    for (int b = 0; b < Chunk<D>::kBoxes; ++b) {
-      pages[b] = -1;
+    for (int b = 0; b < CK::kBoxes; ++b) {
+      rows[b] = 0;
       if (b < nbox) {
         const int pi = (tok0 + b * kBoxRows) >> log2P;
         while (pi >= pid_base + 32) {
@@ -329,71 +354,52 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
           pid_cur = pid_next;
           pid_next = pid_base + 32 + lane < it_npg ? __ldg(ptab + pid_base + 32 + lane) : -1;
         }
-        pages[b] = __shfl_sync(0xffffffffu, pid_cur, pi & 31);
+        int page = __shfl_sync(0xffffffffu, pid_cur, pi & 31);
+        if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) {
+          if (lane == 0) raise_flag(PKV_FLAG_BAD_PAGE);
+          page = 0;
+        }
+        rows[b] = (static_cast<size_t>(page) * p.Hkv + it_g) * p.P + ((tok0 + b * kBoxRows) & (p.P - 1));
       }
     }
+    const uint32_t st = wbase + stage * LY::kStageBytes;
+    const uint16_t* qsrc = p.q + (static_cast<size_t>(it_r) * p.Hq + static_cast<size_t>(it_g) * G) * D;
+    const uint32_t qdst = wbase + LY::kQInOff + it_qslot * (G * D * 2);
+    if (lane == 0) fifo[stage] = ChunkInfo{it_slot, ntok, flags, it_qslot};
     if constexpr (kCpAsync) {
-      // all lanes copy 16-byte pieces; K goes to its swizzled position
-      if (lane == 0) fifo[stage] = ChunkInfo{it_slot, ntok, flags, it_qslot};
       if (ntok > 0) {
-        const uint32_t st = wbase + stage * LY::kStageBytes;
+        constexpr int kPieces = kBoxRows * D / 8;  // 16-byte pieces per 16-row piece
 #pragma unroll
-        for (int b = 0; b < Chunk<D>::kBoxes; ++b) {
+        for (int b = 0; b < CK::kBoxes; ++b) {
           if (b >= nbox) break;
-          int page = pages[b];
-          if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) {
-            if (lane == 0) raise_flag(PKV_FLAG_BAD_PAGE);  // read page 0: wrong values, no stray access
-            page = 0;
-          }
-          const size_t row0 = (static_cast<size_t>(page) * p.Hkv + it_g) * p.P + ((tok0 + b * kBoxRows) & (p.P - 1));
-          const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + row0 * D);
-          const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + row0 * D);
-          constexpr int kPieces = kBoxRows * D / 8;  // 16-byte pieces per 16-row box
+          const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + rows[b] * D);
+          const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + rows[b] * D);
 #pragma unroll
           for (int i = lane; i < kPieces; i += 32) {
-            const int t = i / (D / 8), c16 = i % (D / 8);
-            const int line = (b * kBoxRows + t) * (D / 64) + (c16 >> 3);
-            cp_async16(st + line * 128 + (((c16 & 7) ^ (line & 7)) << 4), ksrc + i * 16);
-            cp_async16(st + LY::kKBytes + ((b * kBoxRows + t) * D + c16 * 8) * 2, vsrc + i * 16);
+            cp_async16(st + b * (kBoxRows * D * 2) + i * 16, ksrc + i * 16);
+            cp_async16(st + LY::kKBytes + b * (kBoxRows * D * 2) + i * 16, vsrc + i * 16);
           }
         }
         if (it_k == 0) {
-          const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(
-              p.q + (static_cast<size_t>(it_r) * p.Hq + static_cast<size_t>(it_g) * G) * D);
-          const uint32_t qdst = wbase + LY::kQInOff + it_qslot * (G * D * 2);
 #pragma unroll
-          for (int i = lane; i < G * D * 2 / 16; i += 32) cp_async16(qdst + i * 16, qsrc + i * 16);
+          for (int i = lane; i < G * D * 2 / 16; i += 32)
+            cp_async16(qdst + i * 16, reinterpret_cast<const uint8_t*>(qsrc) + i * 16);
         }
       }
     } else if (lane == 0) {
-      fifo[stage] = ChunkInfo{it_slot, ntok, flags, it_qslot};
       if (ntok > 0) {
         const bool with_q = it_k == 0;
         const uint32_t bytes = static_cast<uint32_t>(nbox * kBoxRows * D * 2 * 2) +
                                (with_q ? static_cast<uint32_t>(G * D * 2) : 0u);
-        const uint32_t st = wbase + stage * LY::kStageBytes;
         mbar_arrive_expect_tx(full_bar(stage), bytes);
 #pragma unroll
-        for (int b = 0; b < Chunk<D>::kBoxes; ++b) {
+        for (int b = 0; b < CK::kBoxes; ++b) {
           if (b >= nbox) break;
-          int page = pages[b];
-          if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) {
-            raise_flag(PKV_FLAG_BAD_PAGE);  // read page 0 instead: wrong values, no stray access
-            page = 0;
-          }
-          const int row = page * p.Hkv + it_g;
-          const int r0 = (tok0 + b * kBoxRows) & (p.P - 1);
-          // K: one tensor box = 16 token rows x all D/64 parts, swizzled;
-          // V: the same 16 rows are one contiguous run of the pool
-          tma_load_4d(st + b * (kBoxRows * D * 2), &kmap, 0, 0, r0, row, full_bar(stage));
-          bulk_load(st + LY::kKBytes + b * (kBoxRows * D * 2),
-                    p.v_pool + (static_cast<size_t>(row) * p.P + r0) * D, kBoxRows * D * 2,
+          bulk_load(st + b * (kBoxRows * D * 2), p.k_pool + rows[b] * D, kBoxRows * D * 2, full_bar(stage));
+          bulk_load(st + LY::kKBytes + b * (kBoxRows * D * 2), p.v_pool + rows[b] * D, kBoxRows * D * 2,
                     full_bar(stage));
         }
-        if (with_q)
-          bulk_load(wbase + LY::kQInOff + it_qslot * (G * D * 2),
-                    p.q + (static_cast<size_t>(it_r) * p.Hq + static_cast<size_t>(it_g) * G) * D,
-                    G * D * 2, full_bar(stage));
+        if (with_q) bulk_load(qdst, qsrc, G * D * 2, full_bar(stage));
       } else {
         mbar_arrive(full_bar(stage));
       }
@@ -404,10 +410,16 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
   };
 
   // ================================ compute side ================================
-  // token of this lane, and which 64-element part of d it scores
-  const int tl = kLPT == 2 ? (lane & 15) : lane, hh = kLPT == 2 ? (lane >> 4) : 0;
-  float2 o2[G][DPL / 2];
-  float m[G], l[G];
+  // token group tg (token tg of each step), element block i: elements [8i, 8i+8)
+  const int tg = lane / T, ei = lane & (T - 1);
+  const int hl = ei >> (LT - LG);  // the head whose score this lane holds
+  float2 qv[G][4];                 // query * scale*log2(e), elements [8i, 8i+8)
+  float2 o2[G][4];                 // unnormalised output, elements [8i, 8i+8)
+  float m[G];                      // running max per head (log2 units), warp-uniform
+  float m_lane = -INFINITY;        // m[hl]
+  float l_lane = 0.f;              // sum of this lane's weights for head hl
+#pragma unroll
+  for (int g = 0; g < G; ++g) m[g] = -INFINITY;
   // Every issue attempt commits one cp.async group (possibly empty), so the
   // group of chunk n is complete once at most NS-2 newer groups are pending.
   int issued = 0;
@@ -431,20 +443,20 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         m[g] = -INFINITY;
-        l[g] = 0.f;
 #pragma unroll
-        for (int e = 0; e < DPL / 2; ++e) o2[g][e] = make_float2(0.f, 0.f);
+        for (int e = 0; e < 4; ++e) o2[g][e] = make_float2(0.f, 0.f);
       }
+      m_lane = -INFINITY;
+      l_lane = 0.f;
       if (ntok > 0) {
-        // staged bf16 query rows [G][D] -> fp32 pairs [part][32][G][2],
-        // times scale*log2(e)
-        const uint32_t* qin = reinterpret_cast<const uint32_t*>(wb + LY::kQInOff + ci.qslot * (G * D * 2));
-        for (int i = lane; i < G * D / 2; i += 32) {
-          const int g = i / (D / 2), pp = i - g * (D / 2);
-          const int half = pp >> 5, ppl = pp & 31;
-          const uint32_t x = qin[i];
-          *reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(qf) + half * LY::kQHalfBytes + (ppl * G + g) * 8) =
-              make_float2(bf16lo(x) * p.scale_log2, bf16hi(x) * p.scale_log2);
+        const uint8_t* qin = wb + LY::kQInOff + ci.qslot * (G * D * 2) + ei * 16;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const uint4 x = *reinterpret_cast<const uint4*>(qin + g * D * 2);
+          qv[g][0] = make_float2(bf16lo(x.x) * p.scale_log2, bf16hi(x.x) * p.scale_log2);
+          qv[g][1] = make_float2(bf16lo(x.y) * p.scale_log2, bf16hi(x.y) * p.scale_log2);
+          qv[g][2] = make_float2(bf16lo(x.z) * p.scale_log2, bf16hi(x.z) * p.scale_log2);
+          qv[g][3] = make_float2(bf16lo(x.w) * p.scale_log2, bf16hi(x.w) * p.scale_log2);
         }
       }
     }
@@ -459,158 +471,153 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const __grid_co
 
     if (ntok > 0) {
       const uint8_t* stp = wb + stage * LY::kStageBytes;
-      // ---- scores: each lane takes 64 elements (one 128-byte K row) of its token
-      float2 acc[G];
+      const int row_off = (tg * D + ei * 8) * 2;  // this lane's 16 bytes in its token's row
+      const bool partial = ntok < kTok;
+      // ---- scores of every step: lane holds head hl of token step*TPS + tg
+      float sc[STEPS];
 #pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
-      // this lane's 128-byte line of K: token tl, part hh; its swizzle phase
-      // is the line index mod 8
-      const int kline = tl * (D / 64) + hh;
-      const uint8_t* krow = stp + kline * 128;
-      const uint32_t swz = static_cast<uint32_t>(kline & 7) << 4;
-      const uint8_t* qh = reinterpret_cast<const uint8_t*>(qf) + hh * LY::kQHalfBytes;
+      for (int s = 0; s < STEPS; ++s) {
+        const uint4 kk = *reinterpret_cast<const uint4*>(stp + row_off + s * TPS * D * 2);
+        const float2 k0 = make_float2(bf16lo(kk.x), bf16hi(kk.x));
+        const float2 k1 = make_float2(bf16lo(kk.y), bf16hi(kk.y));
+        const float2 k2 = make_float2(bf16lo(kk.z), bf16hi(kk.z));
+        const float2 k3 = make_float2(bf16lo(kk.w), bf16hi(kk.w));
+        float part[G];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 kk = *reinterpret_cast<const uint4*>(krow + ((c << 4) ^ swz));
-        const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
+        for (int g = 0; g < G; ++g) {
+          float2 a = __fmul2_rn(qv[g][0], k0);
+          a = __ffma2_rn(qv[g][1], k1, a);
+          a = __ffma2_rn(qv[g][2], k2, a);
+          a = __ffma2_rn(qv[g][3], k3, a);
+          part[g] = a.x + a.y;
+        }
+        sc[s] = reduce_scatter_heads<G, T>(part, lane);
+      }
+      if (partial) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 k2 = make_float2(bf16lo(kw[j]), bf16hi(kw[j]));
-          const int ppl = c * 4 + j;
-          if constexpr (G == 1) {
-            const float2 q2 = *reinterpret_cast<const float2*>(qh + ppl * 8);
-            acc[0] = __ffma2_rn(q2, k2, acc[0]);
-          } else {
+        for (int s = 0; s < STEPS; ++s)
+          if (s * TPS + tg >= ntok) sc[s] = -INFINITY;
+      }
+      // ---- online softmax (log2 domain).  The running max moves only when a
+      // score exceeds it by more than 2^8; between moves the weights are taken
+      // against the stale max (so p <= 2^8) and the final division by l uses
+      // the same max, so the result is the same softmax.
+      bool grow = false;
 #pragma unroll
-            for (int g = 0; g < G; g += 2) {
-              const float4 q4 = *reinterpret_cast<const float4*>(qh + (ppl * G + g) * 8);
-              acc[g] = __ffma2_rn(make_float2(q4.x, q4.y), k2, acc[g]);
-              acc[g + 1] = __ffma2_rn(make_float2(q4.z, q4.w), k2, acc[g + 1]);
-            }
+      for (int s = 0; s < STEPS; ++s) grow |= sc[s] > m_lane + kLazyRescale;
+      if (__any_sync(0xffffffffu, grow)) {
+        float mx = sc[0];
+#pragma unroll
+        for (int s = 1; s < STEPS; ++s) mx = fmaxf(mx, sc[s]);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float mg = warp_max(hl == g ? mx : -INFINITY);
+          const float mn = fmaxf(m[g], mg);
+          const float alpha = mn == -INFINITY ? 1.f : fast_exp2(m[g] - mn);
+          m[g] = mn;
+          const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o2[g][e] = __fmul2_rn(o2[g][e], a2);
+          if (hl == g) {
+            l_lane *= alpha;
+            m_lane = mn;
           }
         }
       }
-      // ---- online softmax, log2 domain; hidden tokens get -inf -> weight 0.
-      // The running max m is only moved (and o, l rescaled) when some score
-      // exceeds it by more than 2^8 -- in practice on an item's first chunk.
-      // Between moves the exponentials are taken against the stale max, so
-      // p <= 2^8; the final normalisation by l uses the same m, so the
-      // result is the same softmax.
-      float sv[G];
-      bool grow = false;
+      // weights -> per-warp buffer as (p, p) pairs [token][head]
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float x = acc[g].x + acc[g].y;
-        if constexpr (kLPT == 2) x += __shfl_xor_sync(0xffffffffu, x, 16);
-        sv[g] = tl < ntok ? x : -INFINITY;
-        grow |= sv[g] > m[g] + kLazyRescale;
-      }
-      if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float mx = sv[g];
-#pragma unroll
-          for (int o = kTok / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          const float mn = fmaxf(m[g], mx);
-          const float alpha = fast_exp2(m[g] - mn);
-          l[g] *= alpha;
-          const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-          for (int e = 0; e < DPL / 2; ++e) o2[g][e] = __fmul2_rn(o2[g][e], a2);
-          m[g] = mn;
-        }
-      }
-      float pvs[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        pvs[g] = fast_exp2(sv[g] - m[g]);
-        if (hh == 0) l[g] += pvs[g];
-      }
-      if (hh == 0) {
-        if constexpr (G == 1) {
-          *reinterpret_cast<float2*>(pb + tl * 2) = make_float2(pvs[0], pvs[0]);
-        } else {
-#pragma unroll
-          for (int g = 0; g < G; g += 2)
-            *reinterpret_cast<float4*>(pb + (tl * G + g) * 2) = make_float4(pvs[g], pvs[g], pvs[g + 1], pvs[g + 1]);
-        }
+      for (int s = 0; s < STEPS; ++s) {
+        const float pw = fast_exp2(sc[s] - m_lane);
+        l_lane += pw;
+        *reinterpret_cast<float2*>(pb + ((s * TPS + tg) * G + hl) * 2) = make_float2(pw, pw);
       }
       __syncwarp();
-      // ---- P.V: lane owns DPL output columns of every head
-      const uint8_t* vb = stp + LY::kKBytes + lane * DPL * 2;
-      auto pv_token = [&](int t) {
-        float2 pg[G];
-        if constexpr (G == 1) {
-          pg[0] = *reinterpret_cast<const float2*>(pb + t * 2);
-        } else {
+      // ---- P.V: lane accumulates its 8 elements of every head over its tokens
 #pragma unroll
-          for (int g = 0; g < G; g += 2) {
-            const float4 x = *reinterpret_cast<const float4*>(pb + (t * G + g) * 2);
+      for (int s = 0; s < STEPS; ++s) {
+        uint4 vv = *reinterpret_cast<const uint4*>(stp + LY::kKBytes + row_off + s * TPS * D * 2);
+        if (partial && s * TPS + tg >= ntok) vv = make_uint4(0, 0, 0, 0);  // rows past the end may hold anything
+        const float2 v0 = make_float2(bf16lo(vv.x), bf16hi(vv.x));
+        const float2 v1 = make_float2(bf16lo(vv.y), bf16hi(vv.y));
+        const float2 v2 = make_float2(bf16lo(vv.z), bf16hi(vv.z));
+        const float2 v3 = make_float2(bf16lo(vv.w), bf16hi(vv.w));
+        const float* pt = pb + (s * TPS + tg) * G * 2;
+        float2 pg[G];
+#pragma unroll
+        for (int g = 0; g < G; g += 2) {
+          if constexpr (G == 1) {
+            pg[0] = *reinterpret_cast<const float2*>(pt);
+          } else {
+            const float4 x = *reinterpret_cast<const float4*>(pt + g * 2);
             pg[g] = make_float2(x.x, x.y);
             pg[g + 1] = make_float2(x.z, x.w);
           }
         }
-        if constexpr (DPL == 4) {
-          const uint2 x = *reinterpret_cast<const uint2*>(vb + t * D * 2);
-          const float2 v01 = make_float2(bf16lo(x.x), bf16hi(x.x));
-          const float2 v23 = make_float2(bf16lo(x.y), bf16hi(x.y));
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            o2[g][0] = __ffma2_rn(pg[g], v01, o2[g][0]);
-            o2[g][1] = __ffma2_rn(pg[g], v23, o2[g][1]);
-          }
-        } else {
-          const uint32_t x = *reinterpret_cast<const uint32_t*>(vb + t * D * 2);
-          const float2 v01 = make_float2(bf16lo(x), bf16hi(x));
-#pragma unroll
-          for (int g = 0; g < G; ++g) o2[g][0] = __ffma2_rn(pg[g], v01, o2[g][0]);
+        for (int g = 0; g < G; ++g) {
+          o2[g][0] = __ffma2_rn(pg[g], v0, o2[g][0]);
+          o2[g][1] = __ffma2_rn(pg[g], v1, o2[g][1]);
+          o2[g][2] = __ffma2_rn(pg[g], v2, o2[g][2]);
+          o2[g][3] = __ffma2_rn(pg[g], v3, o2[g][3]);
         }
-      };
-      if (ntok == kTok) {  // full chunk: fully unrolled, constant offsets
-#pragma unroll
-        for (int t = 0; t < kTok; ++t) pv_token(t);
-      } else {
-#pragma unroll 1
-        for (int t = 0; t < ntok; ++t) pv_token(t);
       }
+      __syncwarp();  // pb is rewritten by the next chunk
     }
 
     if (ci.flags & kLast) {
-      // ---- item done: normalise and write bf16 output or an fp32 partial
+      // ---- item done: sum the token groups, normalise, and write bf16
+      // output (single-split request) or an fp32 partial and its lse
       const ItemInfo it = items[ci.slot];
 #pragma unroll
+      for (int off = T; off < 32; off <<= 1) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o2[g][e].x += __shfl_xor_sync(0xffffffffu, o2[g][e].x, off);
+            o2[g][e].y += __shfl_xor_sync(0xffffffffu, o2[g][e].y, off);
+          }
+        l_lane += __shfl_xor_sync(0xffffffffu, l_lane, off);
+      }
+#pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float ls = warp_sum(l[g]);
+        const float ls = __shfl_sync(0xffffffffu, l_lane, g << (LT - LG));  // total weight of head g
         const float inv = ls > 0.f ? 1.f / ls : 0.f;
-        const float lse = ls > 0.f ? (m[g] + __log2f(ls)) * 0.69314718055994531f : -INFINITY;
         const size_t row = static_cast<size_t>(it.r) * p.Hq + it.g * G + g;
-        if (it.nsplit == 1) {
-          uint16_t* dst = p.out + row * D + lane * DPL;
-          if constexpr (DPL == 4) {
-            *reinterpret_cast<uint2*>(dst) =
-                make_uint2(pack_bf16x2(o2[g][0].x * inv, o2[g][0].y * inv),
-                           pack_bf16x2(o2[g][1].x * inv, o2[g][1].y * inv));
+        if (tg == 0) {
+          if (it.nsplit == 1) {
+            uint4 w;
+            w.x = pack_bf16x2(o2[g][0].x * inv, o2[g][0].y * inv);
+            w.y = pack_bf16x2(o2[g][1].x * inv, o2[g][1].y * inv);
+            w.z = pack_bf16x2(o2[g][2].x * inv, o2[g][2].y * inv);
+            w.w = pack_bf16x2(o2[g][3].x * inv, o2[g][3].y * inv);
+            *reinterpret_cast<uint4*>(p.out + row * D + ei * 8) = w;
           } else {
-            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(o2[g][0].x * inv, o2[g][0].y * inv);
+            float* dst = p.part_o + (row * p.S_max + it.s) * D + ei * 8;
+            *reinterpret_cast<float4*>(dst) =
+                make_float4(o2[g][0].x * inv, o2[g][0].y * inv, o2[g][1].x * inv, o2[g][1].y * inv);
+            *reinterpret_cast<float4*>(dst + 4) =
+                make_float4(o2[g][2].x * inv, o2[g][2].y * inv, o2[g][3].x * inv, o2[g][3].y * inv);
           }
-          if (p.out_lse != nullptr && lane == 0) p.out_lse[row] = lse;
-        } else {
-          const size_t prow = row * p.S_max + it.s;
-          float* dst = p.part_o + prow * D + lane * DPL;
-          if constexpr (DPL == 4) {
-            *reinterpret_cast<float4*>(dst) = make_float4(o2[g][0].x * inv, o2[g][0].y * inv,
-                                                          o2[g][1].x * inv, o2[g][1].y * inv);
+        }
+        if (lane == 0) {
+          const float lse = ls > 0.f ? (m[g] + __log2f(ls)) * 0.69314718055994531f : -INFINITY;
+          if (it.nsplit == 1) {
+            if (p.out_lse != nullptr) p.out_lse[row] = lse;
           } else {
-            *reinterpret_cast<float2*>(dst) = make_float2(o2[g][0].x * inv, o2[g][0].y * inv);
+            p.part_lse[row * p.S_max + it.s] = lse;
           }
-          if (lane == 0) p.part_lse[prow] = lse;
         }
       }
     }
   }
-  if (n < issued) {
-    // a wait gave up: give copies still in flight a bounded chance to land
-    for (int k = n + 1; k < issued; ++k) mbar_wait(full_bar(k % NS), (k / NS) & 1);
+  if constexpr (!kCpAsync) {
+    if (n < issued) {
+      // a wait gave up: give copies still in flight a bounded chance to land
+      for (int k = n + 1; k < issued; ++k) mbar_wait(full_bar(k % NS), (k / NS) & 1);
+    }
+  } else {
+    cp_async_wait<0>();
   }
   if (lane == 0) {
     __threadfence();

@@ -55,23 +55,6 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 4-D bf16 tensor map over a pool, viewing each token row as D/64 parts of
-// 64 elements: dims (64, D/64, P, pages*Hkv), 128-byte swizzle.
-int make_pool_map_parts(CUtensorMap* map, const void* base, const pkv_pool_desc& pool, uint32_t rows_box) {
-  auto enc = tensor_map_encoder();
-  if (enc == nullptr) return PKV_ERR_TENSOR_MAP;
-  const uint64_t D = pool.head_dim;
-  const cuuint64_t dims[4] = {64, D / 64, static_cast<cuuint64_t>(pool.page_size),
-                              static_cast<cuuint64_t>(pool.num_pages) * pool.num_kv_heads};
-  const cuuint64_t strides[3] = {128, D * 2, static_cast<cuuint64_t>(pool.page_size) * D * 2};
-  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(D / 64), rows_box, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
-                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_TENSOR_MAP;
-}
-
 // 3-D bf16 tensor map: dims[0] innermost (elements), strides in bytes of
 // dims 1 and 2.
 int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
@@ -153,33 +136,35 @@ WorkspaceLayout workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t S) {
 
 // ------------------------------------------------------------ decode launch
 template <int D, int G>
-int launch_decode(const pkv::decode::Params& prm, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                  int sm_count, cudaStream_t stream) {
+int launch_decode(const pkv::decode::Params& prm, int sm_count, cudaStream_t stream) {
 #ifndef PKV_DECODE_NS128
 #define PKV_DECODE_NS128 2
 #endif
 #ifndef PKV_DECODE_NS64
-#define PKV_DECODE_NS64 3
+#define PKV_DECODE_NS64 2
 #endif
 #ifndef PKV_DECODE_MAXW128
-#define PKV_DECODE_MAXW128 10
+#define PKV_DECODE_MAXW128 12
 #endif
 #ifndef PKV_DECODE_MAXW64
 #define PKV_DECODE_MAXW64 12
 #endif
   constexpr int NS = D == 128 ? PKV_DECODE_NS128 : PKV_DECODE_NS64;        // stages per warp
-  constexpr int kMaxW = D == 128 ? PKV_DECODE_MAXW128 : PKV_DECODE_MAXW64;  // warps per CTA
+  // warps per CTA; at G=8 the query and output registers double, so fewer
+  // warps keep every thread's registers unspilled
+  constexpr int kMaxWD = D == 128 ? PKV_DECODE_MAXW128 : PKV_DECODE_MAXW64;
+  constexpr int kMaxW = G == 8 ? (kMaxWD < 10 ? kMaxWD : 10) : kMaxWD;
   using LY = pkv::decode::Layout<D, G, NS>;
   auto kernel = pkv::decode::partition_kernel<D, G, NS, kMaxW>;
   constexpr size_t kBudget = 227 * 1024;
-  const size_t fixed = LY::plan_bytes(prm.B) + 1024;
+  const size_t fixed = LY::bytes(0, prm.B);
   if (fixed + LY::kWarpBytes > kBudget) return PKV_ERR_BAD_SHAPE;  // batch too large for the plan
   const int W = static_cast<int>(std::min<size_t>(kMaxW, (kBudget - fixed) / LY::kWarpBytes));
   const size_t smem = LY::bytes(W, prm.B);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return PKV_ERR_CUDA;
-  kernel<<<sm_count, W * 32, smem, stream>>>(kmap, vmap, prm);
+  kernel<<<sm_count, W * 32, smem, stream>>>(prm);
   if (launch_status() != PKV_OK) return PKV_ERR_CUDA;
   if (prm.partition < 0) return PKV_OK;  // every request is one split
   return launch_combine<D>(prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.S_max, prm.out,
@@ -187,13 +172,12 @@ int launch_decode(const pkv::decode::Params& prm, const CUtensorMap& kmap, const
 }
 
 template <int D>
-int dispatch_decode_group(int group, const pkv::decode::Params& prm, const CUtensorMap& kmap,
-                          const CUtensorMap& vmap, int sm_count, cudaStream_t stream) {
+int dispatch_decode_group(int group, const pkv::decode::Params& prm, int sm_count, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_decode<D, 1>(prm, kmap, vmap, sm_count, stream);
-    case 2: return launch_decode<D, 2>(prm, kmap, vmap, sm_count, stream);
-    case 4: return launch_decode<D, 4>(prm, kmap, vmap, sm_count, stream);
-    case 8: return launch_decode<D, 8>(prm, kmap, vmap, sm_count, stream);
+    case 1: return launch_decode<D, 1>(prm, sm_count, stream);
+    case 2: return launch_decode<D, 2>(prm, sm_count, stream);
+    case 4: return launch_decode<D, 4>(prm, sm_count, stream);
+    case 8: return launch_decode<D, 8>(prm, sm_count, stream);
   }
   return PKV_ERR_UNSUPPORTED;
 }
@@ -321,13 +305,6 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   DeviceInfo dev;
   if ((st = current_device(&dev)) != PKV_OK) return st;
   const int D = pool.head_dim;
-  const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
-  CUtensorMap kmap, vmap;
-  // one box = 16 token rows of one (page, KV head): a page, or half of one
-  if ((st = make_pool_map_parts(&kmap, k_pool, pool, pkv::decode::kBoxRows)) != PKV_OK) return st;
-  if ((st = make_map(&vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, D,
-                     pkv::decode::kBoxRows, 1, false)) != PKV_OK)
-    return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   pkv::decode::Params prm;
   prm.q = static_cast<const uint16_t*>(q);
@@ -351,8 +328,8 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   prm.partition = partition_tokens;
   prm.scale_log2 = scale * 1.4426950408889634f;
   auto s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 128) return dispatch_decode_group<128>(group, prm, kmap, vmap, dev.sm_count, s);
-  return dispatch_decode_group<64>(group, prm, kmap, vmap, dev.sm_count, s);
+  if (D == 128) return dispatch_decode_group<128>(group, prm, dev.sm_count, s);
+  return dispatch_decode_group<64>(group, prm, dev.sm_count, s);
 }
 
 int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
