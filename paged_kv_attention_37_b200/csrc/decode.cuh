@@ -24,20 +24,19 @@
 // cp.async copies from all lanes (or bulk copies issued by one lane).  There
 // is no cross-warp synchronisation after the planning step.
 //
-// Lane layout: T = d/8 lanes share one token, each holding 8 consecutive
-// elements of d, so a warp covers 32/T tokens per step.  The query rows live
-// in registers (fp32, times scale*log2(e)): lane i of a token group keeps
-// elements [8i, 8i+8) of all G heads.  A score is a dot product over the T
-// lanes of a group: a butterfly reduce-scatter over the group leaves each
-// lane with the full score of one head (G partial sums in, one out, no value
-// sent twice).  K and V are each read from shared memory exactly once, with
-// 16-byte loads that cover 512 contiguous bytes per warp (no bank
-// conflicts).  The exponentials go through a small per-warp buffer so that
-// every lane can weight its V elements for all G heads; each lane then
-// accumulates O for its 8 elements x G heads over its tokens, and the token
-// groups are summed with shuffles when the item ends.  The online softmax
-// keeps a warp-uniform running max per head that only moves when a score
-// exceeds it by more than 2^8 (in practice on an item's first chunk).
+// Scores: T lanes share one token (T = 8, or 16 at d=128 with G=8), each
+// holding E = d/T elements of it, so a warp covers 32/T tokens per step.  The
+// query rows live in registers (fp32, times scale*log2(e)): each lane keeps
+// its E elements of all G heads.  A score is a dot product over the T lanes
+// of a group: a butterfly reduce-scatter leaves each lane with the full score
+// of one head (G partial sums in, one out, no value sent twice; the heads are
+// held in a lane-dependent order so the exchange needs no selects).  K is
+// read from shared memory once, with 16-byte loads that cover whole 128-byte
+// lines per quarter warp.  The weights go through a small per-warp buffer;
+// for P.V lane l owns output elements [l*d/32, (l+1)*d/32) of every head and
+// walks the chunk's V rows.  The online softmax keeps a warp-uniform running
+// max per head that only moves when a score exceeds it by more than 2^8 (in
+// practice on an item's first chunk).
 #pragma once
 
 #include "ptx.cuh"
@@ -57,9 +56,6 @@ template <int D>
 struct Chunk {
   static constexpr int kTokens = 2048 / D;             // tokens per pipeline stage (8 KB of K+V)
   static constexpr int kBoxes = kTokens / kBoxRows;    // 16-row pieces per stage (per K or V)
-  static constexpr int kLanesPerToken = D / 8;         // T: each lane holds 8 elements
-  static constexpr int kTokensPerStep = 32 / kLanesPerToken;
-  static constexpr int kSteps = kTokens / kTokensPerStep;
 };
 constexpr int kItemSlots = 8;    // per-warp ring of item descriptors
 constexpr int kMinAutoPartition = 256;
@@ -153,24 +149,22 @@ __device__ __forceinline__ int upper_index(const int32_t* pref, int n, int x) {
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x >> 1); }
 
 // Butterfly reduce-scatter of G per-head partial sums over the T lanes of a
-// token group (T a power of two, lanes [T*k, T*k+T)), then an all-reduce
-// over the group bits left over.  On return v[0] holds the full sum of head
-// (lane & (T-1)) >> (log2 T - log2 G) in every lane.
+// token group (lanes [T*k, T*k+T)), then an all-reduce over the group bits
+// left over.  The caller orders the partial sums per lane as
+// v[j] = head h ^ (G-1-j), h = (lane & (T-1)) >> (log2 T - log2 G): at every
+// level the first half of v is what the partner keeps, so each lane sends
+// v[0..half) and adds what it receives to v[half..G) -- no selects.  On
+// return the result is the full sum of head h.
 template <int G, int T>
-__device__ __forceinline__ float reduce_scatter_heads(float (&v)[G], int lane) {
+__device__ __forceinline__ float reduce_scatter_heads(float (&v)[G]) {
   constexpr int LG = ilog2(G), LT = ilog2(T);
   static_assert(LG <= LT, "more heads than lanes per token");
 #pragma unroll
   for (int lv = 0; lv < LG; ++lv) {
     const int off = T >> (lv + 1);   // partner distance
     const int half = G >> (lv + 1);  // values kept after this level
-    const bool upper = (lane & off) != 0;
 #pragma unroll
-    for (int k = 0; k < half; ++k) {
-      const float send = upper ? v[k] : v[k + half];
-      const float keep = upper ? v[k + half] : v[k];
-      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
+    for (int k = 0; k < half; ++k) v[k] = v[k + half] + __shfl_xor_sync(0xffffffffu, v[k], off);
   }
 #pragma unroll
   for (int off = T >> (LG + 1); off > 0; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
@@ -182,11 +176,15 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   using LY = Layout<D, G, NS>;
   using CK = Chunk<D>;
   constexpr int kTok = CK::kTokens;
-  constexpr int T = CK::kLanesPerToken, TPS = CK::kTokensPerStep, STEPS = CK::kSteps;
+  // score phase: E elements of d per lane (16 at d=128 unless G=8, whose
+  // doubled query registers would not fit; else 8), T lanes per token
+  constexpr int E = (D == 128 && G <= 4) ? 16 : 8;
+  constexpr int T = D / E, TPS = 32 / T, STEPS = kTok / TPS;
   constexpr int LG = ilog2(G), LT = ilog2(T);
+  constexpr int DPL = D / 32;  // P.V output elements per lane
   const int W = blockDim.x >> 5;
   const int log2P = 31 - __clz(p.P);  // P is a power of two
-  static_assert(T == 8 || T == 16, "head_dim 64 or 128");
+  static_assert((T == 8 || T == 16) && (D == 64 || D == 128), "head_dim 64 or 128");
   static_assert(NS >= 2, "at least two stages per warp");
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -410,14 +408,18 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   };
 
   // ================================ compute side ================================
-  // token group tg (token tg of each step), element block i: elements [8i, 8i+8)
+  // Score phase: token group tg (token tg of each step); this lane holds E
+  // elements of d as E/8 pieces of 8, piece j at elements [8*(T*j + ei), +8).
+  // Its query registers hold the G heads in the order perm[j] = h ^ (G-1-j),
+  // h being the head it ends up with, so the reduce-scatter needs no selects.
   const int tg = lane / T, ei = lane & (T - 1);
   const int hl = ei >> (LT - LG);  // the head whose score this lane holds
-  float2 qv[G][4];                 // query * scale*log2(e), elements [8i, 8i+8)
-  float2 o2[G][4];                 // unnormalised output, elements [8i, 8i+8)
+  float2 qv[G][E / 2];             // query * scale*log2(e), permuted heads
+  // P.V phase: lane owns output elements [lane*DPL, (lane+1)*DPL) of every head
+  float2 o2[G][DPL / 2];
   float m[G];                      // running max per head (log2 units), warp-uniform
   float m_lane = -INFINITY;        // m[hl]
-  float l_lane = 0.f;              // sum of this lane's weights for head hl
+  float l_lane = 0.f;              // sum of this lane's weights (head hl, its token group)
 #pragma unroll
   for (int g = 0; g < G; ++g) m[g] = -INFINITY;
   // Every issue attempt commits one cp.async group (possibly empty), so the
@@ -444,19 +446,23 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       for (int g = 0; g < G; ++g) {
         m[g] = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o2[g][e] = make_float2(0.f, 0.f);
+        for (int e = 0; e < DPL / 2; ++e) o2[g][e] = make_float2(0.f, 0.f);
       }
       m_lane = -INFINITY;
       l_lane = 0.f;
       if (ntok > 0) {
         const uint8_t* qin = wb + LY::kQInOff + ci.qslot * (G * D * 2) + ei * 16;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const uint4 x = *reinterpret_cast<const uint4*>(qin + g * D * 2);
-          qv[g][0] = make_float2(bf16lo(x.x) * p.scale_log2, bf16hi(x.x) * p.scale_log2);
-          qv[g][1] = make_float2(bf16lo(x.y) * p.scale_log2, bf16hi(x.y) * p.scale_log2);
-          qv[g][2] = make_float2(bf16lo(x.z) * p.scale_log2, bf16hi(x.z) * p.scale_log2);
-          qv[g][3] = make_float2(bf16lo(x.w) * p.scale_log2, bf16hi(x.w) * p.scale_log2);
+        for (int jj = 0; jj < G; ++jj) {
+          const int head = hl ^ (G - 1 - jj);
+#pragma unroll
+          for (int j = 0; j < E / 8; ++j) {
+            const uint4 x = *reinterpret_cast<const uint4*>(qin + head * D * 2 + j * T * 16);
+            qv[jj][j * 4 + 0] = make_float2(bf16lo(x.x) * p.scale_log2, bf16hi(x.x) * p.scale_log2);
+            qv[jj][j * 4 + 1] = make_float2(bf16lo(x.y) * p.scale_log2, bf16hi(x.y) * p.scale_log2);
+            qv[jj][j * 4 + 2] = make_float2(bf16lo(x.z) * p.scale_log2, bf16hi(x.z) * p.scale_log2);
+            qv[jj][j * 4 + 3] = make_float2(bf16lo(x.w) * p.scale_log2, bf16hi(x.w) * p.scale_log2);
+          }
         }
       }
     }
@@ -471,29 +477,33 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
 
     if (ntok > 0) {
       const uint8_t* stp = wb + stage * LY::kStageBytes;
-      const int row_off = (tg * D + ei * 8) * 2;  // this lane's 16 bytes in its token's row
-      const bool partial = ntok < kTok;
+      const uint8_t* krow = stp + tg * D * 2 + ei * 16;  // piece 0 of this lane's token, step 0
       // ---- scores of every step: lane holds head hl of token step*TPS + tg
       float sc[STEPS];
 #pragma unroll
       for (int s = 0; s < STEPS; ++s) {
-        const uint4 kk = *reinterpret_cast<const uint4*>(stp + row_off + s * TPS * D * 2);
-        const float2 k0 = make_float2(bf16lo(kk.x), bf16hi(kk.x));
-        const float2 k1 = make_float2(bf16lo(kk.y), bf16hi(kk.y));
-        const float2 k2 = make_float2(bf16lo(kk.z), bf16hi(kk.z));
-        const float2 k3 = make_float2(bf16lo(kk.w), bf16hi(kk.w));
+        float2 acc[G];
+#pragma unroll
+        for (int j = 0; j < E / 8; ++j) {
+          const uint4 kk = *reinterpret_cast<const uint4*>(krow + s * TPS * D * 2 + j * T * 16);
+          const float2 k0 = make_float2(bf16lo(kk.x), bf16hi(kk.x));
+          const float2 k1 = make_float2(bf16lo(kk.y), bf16hi(kk.y));
+          const float2 k2 = make_float2(bf16lo(kk.z), bf16hi(kk.z));
+          const float2 k3 = make_float2(bf16lo(kk.w), bf16hi(kk.w));
+#pragma unroll
+          for (int jj = 0; jj < G; ++jj) {
+            float2 a = j == 0 ? __fmul2_rn(qv[jj][0], k0) : __ffma2_rn(qv[jj][j * 4], k0, acc[jj]);
+            a = __ffma2_rn(qv[jj][j * 4 + 1], k1, a);
+            a = __ffma2_rn(qv[jj][j * 4 + 2], k2, a);
+            acc[jj] = __ffma2_rn(qv[jj][j * 4 + 3], k3, a);
+          }
+        }
         float part[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float2 a = __fmul2_rn(qv[g][0], k0);
-          a = __ffma2_rn(qv[g][1], k1, a);
-          a = __ffma2_rn(qv[g][2], k2, a);
-          a = __ffma2_rn(qv[g][3], k3, a);
-          part[g] = a.x + a.y;
-        }
-        sc[s] = reduce_scatter_heads<G, T>(part, lane);
+        for (int jj = 0; jj < G; ++jj) part[jj] = acc[jj].x + acc[jj].y;
+        sc[s] = reduce_scatter_heads<G, T>(part);
       }
-      if (partial) {
+      if (ntok < kTok) {
 #pragma unroll
         for (int s = 0; s < STEPS; ++s)
           if (s * TPS + tg >= ntok) sc[s] = -INFINITY;
@@ -517,7 +527,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
           m[g] = mn;
           const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o2[g][e] = __fmul2_rn(o2[g][e], a2);
+          for (int e = 0; e < DPL / 2; ++e) o2[g][e] = __fmul2_rn(o2[g][e], a2);
           if (hl == g) {
             l_lane *= alpha;
             m_lane = mn;
@@ -532,81 +542,78 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
         *reinterpret_cast<float2*>(pb + ((s * TPS + tg) * G + hl) * 2) = make_float2(pw, pw);
       }
       __syncwarp();
-      // ---- P.V: lane accumulates its 8 elements of every head over its tokens
-#pragma unroll
-      for (int s = 0; s < STEPS; ++s) {
-        uint4 vv = *reinterpret_cast<const uint4*>(stp + LY::kKBytes + row_off + s * TPS * D * 2);
-        if (partial && s * TPS + tg >= ntok) vv = make_uint4(0, 0, 0, 0);  // rows past the end may hold anything
-        const float2 v0 = make_float2(bf16lo(vv.x), bf16hi(vv.x));
-        const float2 v1 = make_float2(bf16lo(vv.y), bf16hi(vv.y));
-        const float2 v2 = make_float2(bf16lo(vv.z), bf16hi(vv.z));
-        const float2 v3 = make_float2(bf16lo(vv.w), bf16hi(vv.w));
-        const float* pt = pb + (s * TPS + tg) * G * 2;
+      // ---- P.V: lane accumulates its DPL elements of every head over the chunk
+      const uint8_t* vb = stp + LY::kKBytes + lane * DPL * 2;
+      auto pv_token = [&](int t) {
         float2 pg[G];
+        if constexpr (G == 1) {
+          pg[0] = *reinterpret_cast<const float2*>(pb + t * 2);
+        } else {
 #pragma unroll
-        for (int g = 0; g < G; g += 2) {
-          if constexpr (G == 1) {
-            pg[0] = *reinterpret_cast<const float2*>(pt);
-          } else {
-            const float4 x = *reinterpret_cast<const float4*>(pt + g * 2);
+          for (int g = 0; g < G; g += 2) {
+            const float4 x = *reinterpret_cast<const float4*>(pb + (t * G + g) * 2);
             pg[g] = make_float2(x.x, x.y);
             pg[g + 1] = make_float2(x.z, x.w);
           }
         }
+        if constexpr (DPL == 4) {
+          const uint2 x = *reinterpret_cast<const uint2*>(vb + t * D * 2);
+          const float2 v01 = make_float2(bf16lo(x.x), bf16hi(x.x));
+          const float2 v23 = make_float2(bf16lo(x.y), bf16hi(x.y));
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          o2[g][0] = __ffma2_rn(pg[g], v0, o2[g][0]);
-          o2[g][1] = __ffma2_rn(pg[g], v1, o2[g][1]);
-          o2[g][2] = __ffma2_rn(pg[g], v2, o2[g][2]);
-          o2[g][3] = __ffma2_rn(pg[g], v3, o2[g][3]);
+          for (int g = 0; g < G; ++g) {
+            o2[g][0] = __ffma2_rn(pg[g], v01, o2[g][0]);
+            o2[g][1] = __ffma2_rn(pg[g], v23, o2[g][1]);
+          }
+        } else {
+          const uint32_t x = *reinterpret_cast<const uint32_t*>(vb + t * D * 2);
+          const float2 v01 = make_float2(bf16lo(x), bf16hi(x));
+#pragma unroll
+          for (int g = 0; g < G; ++g) o2[g][0] = __ffma2_rn(pg[g], v01, o2[g][0]);
         }
+      };
+      if (ntok == kTok) {  // full chunk: fully unrolled, constant offsets
+#pragma unroll
+        for (int t = 0; t < kTok; ++t) pv_token(t);
+      } else {             // rows past ntok may hold anything: never read
+#pragma unroll 1
+        for (int t = 0; t < ntok; ++t) pv_token(t);
       }
       __syncwarp();  // pb is rewritten by the next chunk
     }
 
     if (ci.flags & kLast) {
-      // ---- item done: sum the token groups, normalise, and write bf16
+      // ---- item done: total weight per head, normalise, and write bf16
       // output (single-split request) or an fp32 partial and its lse
       const ItemInfo it = items[ci.slot];
 #pragma unroll
-      for (int off = T; off < 32; off <<= 1) {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            o2[g][e].x += __shfl_xor_sync(0xffffffffu, o2[g][e].x, off);
-            o2[g][e].y += __shfl_xor_sync(0xffffffffu, o2[g][e].y, off);
-          }
-        l_lane += __shfl_xor_sync(0xffffffffu, l_lane, off);
-      }
+      for (int off = T; off < 32; off <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, off);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float ls = __shfl_sync(0xffffffffu, l_lane, g << (LT - LG));  // total weight of head g
         const float inv = ls > 0.f ? 1.f / ls : 0.f;
+        const float lse = ls > 0.f ? (m[g] + __log2f(ls)) * 0.69314718055994531f : -INFINITY;
         const size_t row = static_cast<size_t>(it.r) * p.Hq + it.g * G + g;
-        if (tg == 0) {
-          if (it.nsplit == 1) {
-            uint4 w;
-            w.x = pack_bf16x2(o2[g][0].x * inv, o2[g][0].y * inv);
-            w.y = pack_bf16x2(o2[g][1].x * inv, o2[g][1].y * inv);
-            w.z = pack_bf16x2(o2[g][2].x * inv, o2[g][2].y * inv);
-            w.w = pack_bf16x2(o2[g][3].x * inv, o2[g][3].y * inv);
-            *reinterpret_cast<uint4*>(p.out + row * D + ei * 8) = w;
+        if (it.nsplit == 1) {
+          uint16_t* dst = p.out + row * D + lane * DPL;
+          if constexpr (DPL == 4) {
+            *reinterpret_cast<uint2*>(dst) =
+                make_uint2(pack_bf16x2(o2[g][0].x * inv, o2[g][0].y * inv),
+                           pack_bf16x2(o2[g][1].x * inv, o2[g][1].y * inv));
           } else {
-            float* dst = p.part_o + (row * p.S_max + it.s) * D + ei * 8;
-            *reinterpret_cast<float4*>(dst) =
-                make_float4(o2[g][0].x * inv, o2[g][0].y * inv, o2[g][1].x * inv, o2[g][1].y * inv);
-            *reinterpret_cast<float4*>(dst + 4) =
-                make_float4(o2[g][2].x * inv, o2[g][2].y * inv, o2[g][3].x * inv, o2[g][3].y * inv);
+            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(o2[g][0].x * inv, o2[g][0].y * inv);
           }
-        }
-        if (lane == 0) {
-          const float lse = ls > 0.f ? (m[g] + __log2f(ls)) * 0.69314718055994531f : -INFINITY;
-          if (it.nsplit == 1) {
-            if (p.out_lse != nullptr) p.out_lse[row] = lse;
+          if (p.out_lse != nullptr && lane == 0) p.out_lse[row] = lse;
+        } else {
+          const size_t prow = row * p.S_max + it.s;
+          float* dst = p.part_o + prow * D + lane * DPL;
+          if constexpr (DPL == 4) {
+            *reinterpret_cast<float4*>(dst) = make_float4(o2[g][0].x * inv, o2[g][0].y * inv,
+                                                          o2[g][1].x * inv, o2[g][1].y * inv);
           } else {
-            p.part_lse[row * p.S_max + it.s] = lse;
+            *reinterpret_cast<float2*>(dst) = make_float2(o2[g][0].x * inv, o2[g][0].y * inv);
           }
+          if (lane == 0) p.part_lse[prow] = lse;
         }
       }
     }
