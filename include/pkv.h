@@ -139,19 +139,26 @@ PKV_API size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, in
  *   kv_lens     [batch] int32, keys per request INCLUDING the token appended
  *               this step; 0 gives a zero output (lse -inf)
  *   scale       softmax scale (usually 1/sqrt(d))
- *   partition_tokens  split-K partition length in tokens: 0 = chosen on the
- *               device from the lengths and the SM count; -1 = never split;
- *               otherwise a multiple of 32 in [32, 65536]
+ *   partition_tokens  split-K partition length in tokens: 0 = automatic
+ *               (the batch's token-heads are cut into one equal slice per
+ *               warp of the launch, at least 128 tokens; a request crossing
+ *               slices is merged from partials); -1 = never split; otherwise
+ *               a multiple of 32 in [32, 65536]
  *   workspace   device scratch of pkv_decode_workspace_bytes(...) bytes,
- *               holding split partials and two scheduling counters.  It must
- *               be ZERO-FILLED before its first use; every call leaves the
- *               counters at zero again.  Calls that share a workspace must
- *               not overlap in time.
+ *               holding split partials, two scheduling counters and one
+ *               finished-split counter per (request, KV head).  It must be
+ *               ZERO-FILLED before its first use; every call that completes
+ *               leaves the counters at zero again (after a call that raised
+ *               PKV_FLAG_WAIT_TIMEOUT, zero it again).  Calls that share a
+ *               workspace must not overlap in time.
  *   out         [batch][Hq][d] bf16 (written)
  *   out_lse     [batch][Hq] fp32 natural-log softmax denominators, or NULL
  *
- * Requests whose length fits one partition are written by the partition
- * kernel directly; the others go through partials and the combine kernel.
+ * Requests that are not split are written by the partition kernel directly.
+ * Split ones go through fp32 partials: with the automatic split, a (request,
+ * KV head) cut into at most 8 pieces is merged inside the partition kernel by
+ * the warp finishing its last piece, longer ones (and every split request of
+ * a fixed partition) by a second, combine kernel.
  */
 PKV_API int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads,
                           const void* k_pool, const void* v_pool, pkv_pool_desc pool,

@@ -9,12 +9,20 @@
 // mini-vllm advanced series design, section 4 Phase B adv04 (split-K over a
 // long KV sequence).
 //
-// Work unit ("item"): one (request r, KV head g, split s); it covers tokens
-// [s*part, min((s+1)*part, L_r)) and produces the outputs of all G query
-// heads of the group, so every K/V byte is read from HBM once and used G
-// times.  Items whose length is a whole partition are handed out first, the
-// shorter remainders last (largest-first order), from an atomic counter in
-// the workspace (dynamic load balancing over ragged lengths).
+// Work unit ("item"): a token range of one (request r, KV head g); it
+// produces the outputs of all G query heads of the group, so every K/V byte
+// is read from HBM once and used G times.  Two schedules:
+//   automatic split (partition_tokens == 0): each group is padded to whole
+//   32-token quanta and the groups are laid end to end; warp w takes the
+//   w-th equal slice (at least kMinShare tokens) of that line, so every warp
+//   streams the same number of bytes and all finish together.  A slice may
+//   end inside a group and the next one continue it: such a group's pieces
+//   are split-K partials, merged by the warp that finishes the group's last
+//   piece (at most kFusedMergeMax pieces) or by combine_kernel (more).
+//   fixed partition: items are (r, g, split s) of the given length; whole
+//   partitions are handed out first and the shorter remainders last, from an
+//   atomic counter in the workspace (dynamic balancing over ragged lengths),
+//   and combine_kernel merges the partials.
 //
 // Every warp is independent: it takes an item, walks its page-table entries
 // (32 per warp-wide load), and keeps NS-1 chunks in flight in its own ring of
@@ -58,11 +66,17 @@ struct Chunk {
   static constexpr int kBoxes = kTokens / kBoxRows;    // 16-row pieces per stage (per K or V)
 };
 constexpr int kItemSlots = 8;    // per-warp ring of item descriptors
-constexpr int kMinAutoPartition = 256;
-constexpr int kMaxAutoPartition = 8192;
-constexpr int kAutoItemsPerWarp = 3;  // auto split: each warp's share >= 3 partitions
+// Automatic split (partition_tokens == 0): the padded token-heads of the
+// batch are cut into one equal slice per warp, at least kMinShare tokens, so
+// every warp streams the same number of bytes and all finish together.
+constexpr int kMinShare = 128;
 
 constexpr int kPartitionQuantum = 32;  // split lengths are multiples of this
+// A (request, KV head) group cut into at most this many splits is merged
+// inside the partition kernel by the warp that finishes its last split;
+// groups with more splits are merged by combine_kernel, whose CTAs spread the
+// partial reads over many SMs.
+constexpr int kFusedMergeMax = 8;
 constexpr float kLazyRescale = 8.0f;  // log2 units: move the running max when it grows > 2^8
 constexpr int kFirst = 1;  // first chunk of an item
 constexpr int kLast = 2;   // last chunk of an item
@@ -79,6 +93,8 @@ struct Params {
   float* part_lse;            // [B][Hq][S_max]
   int32_t* num_splits;        // [B]
   uint32_t* counters;         // [0] next item, [1] finished warps
+  uint32_t* group_done;       // [B*Hkv] splits finished per (request, KV head) (automatic split)
+  int32_t* group_splits;      // [B*Hkv] splits of each (request, KV head) (automatic split)
   int32_t B, Hq, Hkv, P, max_pages, num_pages, S_max, partition;
   float scale_log2;           // softmax scale * log2(e)
 };
@@ -171,6 +187,71 @@ __device__ __forceinline__ float reduce_scatter_heads(float (&v)[G]) {
   return v[0];
 }
 
+// Merge the nsplit partials of the G query heads of one (request, KV head)
+// group: o = sum_s w_s o_s / sum_s w_s with w_s = exp(lse_s - max lse) (the
+// split-K rule of combine_kernel).  One warp; lane l owns output elements
+// [l*D/32, (l+1)*D/32).  Partials are read through L2 (other warps wrote them
+// during this launch), all splits of a head in one batch of loads, so a merge
+// costs about one memory round trip per head.  nsplit <= kFusedMergeMax.
+template <int D, int G>
+__device__ __forceinline__ void merge_group(const Params& p, int r, int g, int nsplit, int lane) {
+  constexpr int DPL = D / 32;
+  constexpr int HB = 1;  // heads per batch of loads
+  constexpr float kLog2e = 1.4426950408889634f;
+  const size_t row0 = static_cast<size_t>(r) * p.Hq + static_cast<size_t>(g) * G;
+  float ls[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+    ls[h] = lane < nsplit ? __ldcg(p.part_lse + (row0 + h) * p.S_max + lane) : -INFINITY;
+#pragma unroll
+  for (int h0 = 0; h0 < G; h0 += HB) {
+    float v[HB][kFusedMergeMax][DPL];
+#pragma unroll
+    for (int hb = 0; hb < HB; ++hb) {
+      const float* po = p.part_o + (row0 + h0 + hb) * p.S_max * D + lane * DPL;
+#pragma unroll
+      for (int s = 0; s < kFusedMergeMax; ++s) {
+        if (s < nsplit) {
+          if constexpr (DPL == 4) {
+            const float4 x = __ldcg(reinterpret_cast<const float4*>(po + static_cast<size_t>(s) * D));
+            v[hb][s][0] = x.x; v[hb][s][1] = x.y; v[hb][s][2] = x.z; v[hb][s][3] = x.w;
+          } else {
+            const float2 x = __ldcg(reinterpret_cast<const float2*>(po + static_cast<size_t>(s) * D));
+            v[hb][s][0] = x.x; v[hb][s][1] = x.y;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int hb = 0; hb < HB; ++hb) {
+      const int h = h0 + hb;
+      const float M = warp_max(ls[h]);
+      const float w = M == -INFINITY ? 0.f : fast_exp2((ls[h] - M) * kLog2e);
+      const float den = warp_sum(w);
+      float acc[DPL];
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int s = 0; s < kFusedMergeMax; ++s) {
+        const float ws = __shfl_sync(0xffffffffu, w, s);
+        if (s < nsplit) {
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(ws, v[hb][s][e], acc[e]);
+        }
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      uint16_t* dst = p.out + (row0 + h) * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        *reinterpret_cast<uint2*>(dst) =
+            make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      }
+      if (p.out_lse != nullptr && lane == 0) p.out_lse[row0 + h] = den > 0.f ? M + logf(den) : -INFINITY;
+    }
+  }
+}
+
 template <int D, int G, int NS, int MAXW>
 __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p) {
   using LY = Layout<D, G, NS>;
@@ -208,13 +289,16 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     }
   }
 
-  // ---- plan (warp 0): clamp lengths, pick the partition, count the items:
-  // whole-partition items first (prefF), then one remainder item per
-  // (request, KV head) whose length is not a multiple of the partition
-  // (prefR; an empty request also gets one, to write its zero output).
+  // ---- plan (warp 0).  Automatic split: every (request, KV head) group is
+  // padded to whole 32-token quanta (an empty request to one, so its zero
+  // output is written); prefF[r] is the first quantum of request r's groups
+  // in the concatenation, and warp w takes quanta [w*share, (w+1)*share).
+  // Fixed partition: whole-partition items first (prefF), then one remainder
+  // item per (request, KV head) whose length is not a multiple of the
+  // partition (prefR; an empty request also gets one).
+  const bool balanced = p.partition == 0;
   if (warp == 0) {
     const int maxL = p.max_pages * p.P;
-    long long tot = 0;
     bool bad = false;
     for (int r = lane; r < p.B; r += 32) {
       int L = p.kv_lens[r];
@@ -223,25 +307,39 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
         L = L < 0 ? 0 : maxL;
       }
       lens[r] = L;
-      tot += L;
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) raise_flag(PKV_FLAG_BAD_LENGTH);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    int part;
+    int part = 0;
     if (p.partition > 0) {
       part = p.partition;
     } else if (p.partition < 0) {
       part = ((maxL > 0 ? maxL : 1) + kPartitionQuantum - 1) / kPartitionQuantum * kPartitionQuantum;
-    } else {
-      const long long warps = static_cast<long long>(gridDim.x) * W;
-      const long long share = tot * p.Hkv / (warps * kAutoItemsPerWarp);
-      part = kMaxAutoPartition;
-      while (part > kMinAutoPartition && part > share) part >>= 1;
     }
     __syncwarp();
     int runF = 0, runR = 0;
-    for (int base = 0; base < p.B; base += 32) {
+    if (balanced) {
+      for (int base = 0; base < p.B; base += 32) {
+        const int r = base + lane;
+        int nq = 0;
+        if (r < p.B) nq = max(1, (lens[r] + kPartitionQuantum - 1) / kPartitionQuantum) * p.Hkv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, nq, o);
+          if (lane >= o) nq += y;
+        }
+        if (r < p.B) prefF[r + 1] = runF + nq;
+        runF += __shfl_sync(0xffffffffu, nq, 31);
+      }
+      const long long warps = static_cast<long long>(gridDim.x) * W;
+      const int share = max(kMinShare / kPartitionQuantum, static_cast<int>((runF + warps - 1) / warps));
+      if (lane == 0) {
+        prefF[0] = 0;
+        misc[0] = share;  // quanta per warp
+        misc[1] = runF;   // total quanta
+        misc[2] = 0;
+      }
+    }
+    for (int base = 0; base < p.B && !balanced; base += 32) {
       const int r = base + lane;
       int nf = 0, nr = 0;
       if (r < p.B) {
@@ -266,7 +364,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       runF += __shfl_sync(0xffffffffu, nf, 31);
       runR += __shfl_sync(0xffffffffu, nr, 31);
     }
-    if (lane == 0) {
+    if (lane == 0 && !balanced) {
       prefF[0] = 0;
       prefR[0] = 0;
       misc[0] = part;
@@ -276,6 +374,10 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   }
   __syncthreads();
   const int part = misc[0], nF = misc[1], total = misc[1] + misc[2];
+  // automatic split: this warp's quanta [bq, bq_end), share = misc[0]
+  const int wid = blockIdx.x * W + warp;
+  int bq = balanced ? static_cast<int>(min(static_cast<long long>(wid) * part, static_cast<long long>(nF))) : 0;
+  const int bq_end = balanced ? static_cast<int>(min(static_cast<long long>(wid + 1) * part, static_cast<long long>(nF))) : 0;
 
   // ================= issue side: item cursor, lane 0 issues TMA =================
   bool more = true, active = false;
@@ -284,6 +386,24 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   const int32_t* ptab = p.page_table;
 
   auto fetch = [&]() {
+    int r, g, s, t0, ntok, nsplit;
+    if (balanced) {
+      // next piece of this warp's slice: the rest of the group at bq
+      if (bq >= bq_end) {
+        more = false;
+        return;
+      }
+      r = upper_index(prefF, p.B, bq);
+      const int gq = (prefF[r + 1] - prefF[r]) / p.Hkv;  // quanta per group of request r
+      g = (bq - prefF[r]) / gq;
+      const int gstart = prefF[r] + g * gq, gend = gstart + gq;
+      const int iend = min(gend, bq_end);
+      t0 = (bq - gstart) * kPartitionQuantum;
+      ntok = max(0, min((iend - gstart) * kPartitionQuantum, lens[r]) - t0);
+      s = wid - gstart / part;
+      nsplit = (gend - 1) / part - gstart / part + 1;
+      bq = iend;
+    } else {
     int idx = 0;
     if (lane == 0) idx = static_cast<int>(atomicAdd(p.counters, 1u));
     idx = __shfl_sync(0xffffffffu, idx, 0);
@@ -291,7 +411,6 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       more = false;
       return;
     }
-    int r, g, s, t0, ntok;
     if (idx < nF) {
       r = upper_index(prefF, p.B, idx);
       const int local = idx - prefF[r];
@@ -307,7 +426,8 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       t0 = s * part;
       ntok = lens[r] - t0;
     }
-    const int L = lens[r];
+    nsplit = lens[r] == 0 ? 1 : (lens[r] + part - 1) / part;
+    }
     it_r = r;
     it_g = g;
     it_t0 = t0;
@@ -317,7 +437,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     it_slot = fetched % kItemSlots;
     it_qslot = fetched % NS;
     ++fetched;
-    if (lane == 0) items[it_slot] = ItemInfo{r, g, s, L == 0 ? 1 : (L + part - 1) / part};
+    if (lane == 0) items[it_slot] = ItemInfo{r, g, s, nsplit};
     it_npg = (ntok + p.P - 1) >> log2P;
     ptab = p.page_table + static_cast<size_t>(r) * p.max_pages + (t0 >> log2P);
     pid_base = 0;
@@ -616,6 +736,25 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
           if (lane == 0) p.part_lse[prow] = lse;
         }
       }
+      if (balanced && it.nsplit > 1) {
+        const size_t gi = static_cast<size_t>(it.r) * p.Hkv + it.g;
+        if (it.s == 0 && lane == 0) p.group_splits[gi] = it.nsplit;
+        if (it.nsplit <= kFusedMergeMax) {
+          // the warp that finishes the group's last split merges the partials
+          __threadfence();
+          __syncwarp();
+          uint32_t done = 0;
+          if (lane == 0) done = atomicAdd(p.group_done + gi, 1u);
+          done = __shfl_sync(0xffffffffu, done, 0);
+          if (done == static_cast<uint32_t>(it.nsplit - 1)) {
+            __threadfence();
+            merge_group<D, G>(p, it.r, it.g, it.nsplit, lane);
+            if (lane == 0) p.group_done[gi] = 0;  // ready for the next launch
+          }
+        }
+      } else if (balanced && it.s == 0 && lane == 0) {
+        p.group_splits[static_cast<size_t>(it.r) * p.Hkv + it.g] = 1;
+      }
     }
   }
   if constexpr (!kCpAsync) {
@@ -639,23 +778,25 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
 // Merge split partials.  One CTA per (request, query head) row; its warps
 // stride over the splits (four splits' loads in flight per warp), each lane
 // owning D/32 columns, and the per-warp sums meet in shared memory.
-// skip_single: requests with one split were written by the partition kernel.
+// num_splits[row / rows_per_entry] is the row's split count (per request in
+// the standalone combine, per (request, KV head) group after an automatic
+// split); rows with at most skip_below splits are left alone (written by the
+// partition kernel).
 constexpr int kCombineMaxWarps = 8;
 
 template <int D>
 __global__ void __launch_bounds__(32 * kCombineMaxWarps) combine_kernel(
     const float* __restrict__ part_o, const float* __restrict__ part_lse,
-    const int32_t* __restrict__ num_splits, int32_t B, int32_t Hq, int32_t S_max,
-    uint16_t* __restrict__ out, float* __restrict__ out_lse, int skip_single) {
+    const int32_t* __restrict__ num_splits, int32_t rows_per_entry, int32_t S_max,
+    uint16_t* __restrict__ out, float* __restrict__ out_lse, int skip_below) {
   constexpr int DPL = D / 32;
   constexpr float kLog2e = 1.4426950408889634f;
   __shared__ float red_m[kCombineMaxWarps], red_den[kCombineMaxWarps];
   __shared__ __align__(16) float red_acc[kCombineMaxWarps][D];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const long long row = blockIdx.x;
-  const int r = static_cast<int>(row / Hq);
-  int n = num_splits[r];
-  if (skip_single && n <= 1) return;
+  int n = num_splits[row / rows_per_entry];
+  if (n <= skip_below) return;
   n = max(0, min(n, S_max));
   const float* ls = part_lse + row * S_max;
   float M = -INFINITY;

@@ -103,32 +103,45 @@ int combine_warps(int32_t max_splits) {
 
 template <int D>
 int launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits, int32_t B,
-                   int32_t Hq, int32_t S, uint16_t* out, float* out_lse, int skip_single,
-                   cudaStream_t stream) {
+                   int32_t Hq, int32_t rows_per_entry, int32_t S, uint16_t* out, float* out_lse,
+                   int skip_below, cudaStream_t stream) {
   const long long rows = static_cast<long long>(B) * Hq;
   if (rows > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
   pkv::decode::combine_kernel<D><<<static_cast<unsigned>(rows), 32 * combine_warps(S), 0, stream>>>(
-      part_o, part_lse, num_splits, B, Hq, S, out, out_lse, skip_single);
+      part_o, part_lse, num_splits, rows_per_entry, S, out, out_lse, skip_below);
   return launch_status();
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Partial slots per (request, query head): a fixed partition gives
+// ceil(len / partition) splits; the automatic split gives a group of padded
+// length Lp at most ceil(Lp / kMinShare) + 1 (slices are >= kMinShare tokens,
+// and the group's first and last slice may be partial).
 int32_t max_splits_for(int32_t max_kv_len, int32_t partition_tokens) {
   if (partition_tokens < 0) return 1;
-  const int32_t part = partition_tokens > 0 ? partition_tokens : pkv::decode::kMinAutoPartition;
-  return std::max<int32_t>(1, (std::max<int32_t>(max_kv_len, 1) + part - 1) / part);
+  const int32_t len = std::max<int32_t>(max_kv_len, 1);
+  if (partition_tokens == 0) return (len + pkv::decode::kMinShare - 1) / pkv::decode::kMinShare + 1;
+  return (len + partition_tokens - 1) / partition_tokens;
 }
 
+// Workspace: [counters | group_done | num_splits | group_splits | part_lse |
+// part_o].  The first two regions must be zero before the first call; every
+// call that completes leaves them zero (zero_bytes covers them).
 struct WorkspaceLayout {
-  size_t counters = 0, num_splits = 0, part_lse = 0, part_o = 0, total = 0;
+  size_t counters = 0, group_done = 0, num_splits = 0, group_splits = 0, part_lse = 0, part_o = 0,
+         total = 0, zero_bytes = 0;
 };
 
 WorkspaceLayout workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t S) {
   WorkspaceLayout w;
+  const size_t groups = static_cast<size_t>(B) * Hq;  // Hq bounds the KV heads
   w.counters = 0;
-  w.num_splits = 256;
-  w.part_lse = w.num_splits + align256(static_cast<size_t>(B) * 4);
+  w.group_done = 256;
+  w.num_splits = w.group_done + align256(groups * 4);
+  w.zero_bytes = w.num_splits;
+  w.group_splits = w.num_splits + align256(static_cast<size_t>(B) * 4);
+  w.part_lse = w.group_splits + align256(groups * 4);
   w.part_o = w.part_lse + align256(static_cast<size_t>(B) * Hq * S * 4);
   w.total = w.part_o + align256(static_cast<size_t>(B) * Hq * S * D * 4);
   return w;
@@ -153,7 +166,7 @@ int launch_decode(const pkv::decode::Params& prm, int sm_count, cudaStream_t str
   // warps per CTA; at G=8 the query and output registers double, so fewer
   // warps keep every thread's registers unspilled
   constexpr int kMaxWD = D == 128 ? PKV_DECODE_MAXW128 : PKV_DECODE_MAXW64;
-  constexpr int kMaxW = G == 8 ? (kMaxWD < 10 ? kMaxWD : 10) : kMaxWD;
+  constexpr int kMaxW = G == 8 ? (kMaxWD < 8 ? kMaxWD : 8) : kMaxWD;
   using LY = pkv::decode::Layout<D, G, NS>;
   auto kernel = pkv::decode::partition_kernel<D, G, NS, kMaxW>;
   constexpr size_t kBudget = 227 * 1024;
@@ -167,8 +180,15 @@ int launch_decode(const pkv::decode::Params& prm, int sm_count, cudaStream_t str
   kernel<<<sm_count, W * 32, smem, stream>>>(prm);
   if (launch_status() != PKV_OK) return PKV_ERR_CUDA;
   if (prm.partition < 0) return PKV_OK;  // every request is one split
-  return launch_combine<D>(prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.S_max, prm.out,
-                           prm.out_lse, 1, stream);
+  if (prm.partition == 0) {
+    // automatic split: groups of at most kFusedMergeMax splits were merged in
+    // the partition kernel; the combine kernel takes the longer ones
+    if (prm.S_max <= pkv::decode::kFusedMergeMax) return PKV_OK;
+    return launch_combine<D>(prm.part_o, prm.part_lse, prm.group_splits, prm.B, prm.Hq, G, prm.S_max,
+                             prm.out, prm.out_lse, pkv::decode::kFusedMergeMax, stream);
+  }
+  return launch_combine<D>(prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.Hq, prm.S_max,
+                           prm.out, prm.out_lse, 1, stream);
 }
 
 template <int D>
@@ -298,6 +318,11 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
     return PKV_ERR_MISALIGNED;
   const int32_t max_kv = max_pages * pool.page_size;
+  // the automatic split counts the batch's token-heads in 32-token quanta (int32)
+  if (partition_tokens == 0 &&
+      static_cast<long long>(batch) * pool.num_kv_heads * (max_kv / pkv::decode::kPartitionQuantum + 1) >=
+          (1ll << 31))
+    return PKV_ERR_BAD_SHAPE;
   const int32_t S = max_splits_for(max_kv, partition_tokens);
   const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, pool.head_dim, S);
   if (workspace == nullptr || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
@@ -318,6 +343,8 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   prm.part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
   prm.num_splits = reinterpret_cast<int32_t*>(ws + wl.num_splits);
   prm.counters = reinterpret_cast<uint32_t*>(ws + wl.counters);
+  prm.group_done = reinterpret_cast<uint32_t*>(ws + wl.group_done);
+  prm.group_splits = reinterpret_cast<int32_t*>(ws + wl.group_splits);
   prm.B = batch;
   prm.Hq = num_q_heads;
   prm.Hkv = pool.num_kv_heads;
@@ -345,10 +372,10 @@ int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_
   if ((st = current_device(&dev)) != PKV_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if (head_dim == 128)
-    return launch_combine<128>(part_o, part_lse, num_splits, batch, num_q_heads, max_splits,
-                               static_cast<uint16_t*>(out), out_lse, 0, s);
-  return launch_combine<64>(part_o, part_lse, num_splits, batch, num_q_heads, max_splits,
-                            static_cast<uint16_t*>(out), out_lse, 0, s);
+    return launch_combine<128>(part_o, part_lse, num_splits, batch, num_q_heads, num_q_heads, max_splits,
+                               static_cast<uint16_t*>(out), out_lse, -1, s);
+  return launch_combine<64>(part_o, part_lse, num_splits, batch, num_q_heads, num_q_heads, max_splits,
+                            static_cast<uint16_t*>(out), out_lse, -1, s);
 }
 
 int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch,
@@ -483,9 +510,13 @@ extern "C" int pkv_paged_attn_decode_static(const void* q, int32_t batch, int32_
   if (batch == 0) return PKV_OK;
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != PKV_OK) return st;
-  // The array keeps whatever the previous call left; the scheduling counters
-  // at its start must be zero when the decode kernel begins.
-  if (cudaMemsetAsync(scratch, 0, 256, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // The array keeps whatever the previous call left; the scheduling and
+  // per-group split counters at its start must be zero when the decode
+  // kernel begins.
+  const size_t zero = workspace_layout(batch, num_q_heads, pool.head_dim,
+                                       max_splits_for(static_cast<int32_t>(max_kv), partition_tokens))
+                          .zero_bytes;
+  if (cudaMemsetAsync(scratch, 0, zero, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return PKV_ERR_CUDA;
   return pkv_paged_attn_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages,
                                kv_lens, scale, partition_tokens, scratch, kStaticScratchBytes, out,
