@@ -373,6 +373,9 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     }
   }
   __syncthreads();
+  // let a dependent launch (the combine kernel) be scheduled now; it waits
+  // for this whole grid to finish before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int part = misc[0], nF = misc[1], total = misc[1] + misc[2];
   // automatic split: this warp's quanta [bq, bq_end), share = misc[0]
   const int wid = blockIdx.x * W + warp;
@@ -795,6 +798,9 @@ __global__ void __launch_bounds__(32 * kCombineMaxWarps) combine_kernel(
   __shared__ __align__(16) float red_acc[kCombineMaxWarps][D];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const long long row = blockIdx.x;
+  // launched as a programmatic dependent of the partition kernel: wait for
+  // that grid to complete (a no-op when launched normally)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   int n = num_splits[row / rows_per_entry];
   if (n <= skip_below) return;
   n = max(0, min(n, S_max));

@@ -101,14 +101,30 @@ int combine_warps(int32_t max_splits) {
   return w;
 }
 
+// after_decode: the combine follows the partition kernel on the stream and is
+// launched as its programmatic dependent (the partition kernel signals at its
+// start, the combine waits for the partition grid's completion before its
+// first read), so the combine's launch overlaps the partition kernel instead
+// of following its last CTA.
 template <int D>
 int launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits, int32_t B,
                    int32_t Hq, int32_t rows_per_entry, int32_t S, uint16_t* out, float* out_lse,
-                   int skip_below, cudaStream_t stream) {
+                   int skip_below, bool after_decode, cudaStream_t stream) {
   const long long rows = static_cast<long long>(B) * Hq;
   if (rows > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
-  pkv::decode::combine_kernel<D><<<static_cast<unsigned>(rows), 32 * combine_warps(S), 0, stream>>>(
-      part_o, part_lse, num_splits, rows_per_entry, S, out, out_lse, skip_below);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows));
+  cfg.blockDim = dim3(32 * combine_warps(S));
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_decode ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, pkv::decode::combine_kernel<D>, part_o, part_lse, num_splits, rows_per_entry, S,
+                         out, out_lse, skip_below) != cudaSuccess)
+    return PKV_ERR_CUDA;
   return launch_status();
 }
 
@@ -185,10 +201,10 @@ int launch_decode(const pkv::decode::Params& prm, int sm_count, cudaStream_t str
     // the partition kernel; the combine kernel takes the longer ones
     if (prm.S_max <= pkv::decode::kFusedMergeMax) return PKV_OK;
     return launch_combine<D>(prm.part_o, prm.part_lse, prm.group_splits, prm.B, prm.Hq, G, prm.S_max,
-                             prm.out, prm.out_lse, pkv::decode::kFusedMergeMax, stream);
+                             prm.out, prm.out_lse, pkv::decode::kFusedMergeMax, true, stream);
   }
   return launch_combine<D>(prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.Hq, prm.S_max,
-                           prm.out, prm.out_lse, 1, stream);
+                           prm.out, prm.out_lse, 1, true, stream);
 }
 
 template <int D>
@@ -373,9 +389,9 @@ int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if (head_dim == 128)
     return launch_combine<128>(part_o, part_lse, num_splits, batch, num_q_heads, num_q_heads, max_splits,
-                               static_cast<uint16_t*>(out), out_lse, -1, s);
+                               static_cast<uint16_t*>(out), out_lse, -1, false, s);
   return launch_combine<64>(part_o, part_lse, num_splits, batch, num_q_heads, num_q_heads, max_splits,
-                            static_cast<uint16_t*>(out), out_lse, -1, s);
+                            static_cast<uint16_t*>(out), out_lse, -1, false, s);
 }
 
 int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch,
