@@ -14,8 +14,9 @@
 // is read from HBM once and used G times.  Two schedules:
 //   automatic split (partition_tokens == 0): each group is padded to whole
 //   32-token quanta and the groups are laid end to end; warp w takes the
-//   w-th equal slice (at least kMinShare tokens) of that line, so every warp
-//   streams the same number of bytes and all finish together.  A slice may
+//   w-th of Weff equal slices (to one quantum; at least kMinShare tokens) of
+//   that line, so every warp streams the same number of bytes and all finish
+//   together.  A slice may
 //   end inside a group and the next one continue it: such a group's pieces
 //   are split-K partials, merged by the warp that finishes the group's last
 //   piece (at most kFusedMergeMax pieces) or by combine_kernel (more).
@@ -330,12 +331,13 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
         if (r < p.B) prefF[r + 1] = runF + nq;
         runF += __shfl_sync(0xffffffffu, nq, 31);
       }
-      const long long warps = static_cast<long long>(gridDim.x) * W;
-      const int share = max(kMinShare / kPartitionQuantum, static_cast<int>((runF + warps - 1) / warps));
+      // slices of floor(Q/Weff) or one quantum more, at least kMinShare tokens
+      const int weff = static_cast<int>(
+          min(static_cast<long long>(gridDim.x) * W, max(1ll, static_cast<long long>(runF) / (kMinShare / kPartitionQuantum))));
       if (lane == 0) {
         prefF[0] = 0;
-        misc[0] = share;  // quanta per warp
-        misc[1] = runF;   // total quanta
+        misc[0] = weff;  // warps with a slice
+        misc[1] = runF;  // total quanta
         misc[2] = 0;
       }
     }
@@ -377,10 +379,14 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   // for this whole grid to finish before reading anything
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int part = misc[0], nF = misc[1], total = misc[1] + misc[2];
-  // automatic split: this warp's quanta [bq, bq_end), share = misc[0]
+  // automatic split: warp w < Weff (= misc[0]) takes quanta
+  // [floor(w*Q/Weff), floor((w+1)*Q/Weff)); the slice holding quantum x is
+  // floor(((x+1)*Weff - 1) / Q)
   const int wid = blockIdx.x * W + warp;
-  int bq = balanced ? static_cast<int>(min(static_cast<long long>(wid) * part, static_cast<long long>(nF))) : 0;
-  const int bq_end = balanced ? static_cast<int>(min(static_cast<long long>(wid + 1) * part, static_cast<long long>(nF))) : 0;
+  auto slice_start = [&](int w) { return static_cast<int>(static_cast<long long>(w) * nF / part); };
+  auto slice_of = [&](int x) { return static_cast<int>((static_cast<long long>(x + 1) * part - 1) / nF); };
+  int bq = balanced && wid < part ? slice_start(wid) : 0;
+  const int bq_end = balanced && wid < part ? slice_start(wid + 1) : 0;
 
   // ================= issue side: item cursor, lane 0 issues TMA =================
   bool more = true, active = false;
@@ -403,8 +409,8 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       const int iend = min(gend, bq_end);
       t0 = (bq - gstart) * kPartitionQuantum;
       ntok = max(0, min((iend - gstart) * kPartitionQuantum, lens[r]) - t0);
-      s = wid - gstart / part;
-      nsplit = (gend - 1) / part - gstart / part + 1;
+      s = wid - slice_of(gstart);
+      nsplit = slice_of(gend - 1) - slice_of(gstart) + 1;
       bq = iend;
     } else {
     int idx = 0;
