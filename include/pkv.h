@@ -147,9 +147,13 @@ PKV_API size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, in
  *   workspace   device scratch of pkv_decode_workspace_bytes(...) bytes,
  *               holding split partials, two scheduling counters and one
  *               finished-split counter per (request, KV head).  It must be
- *               ZERO-FILLED before its first use; every call that completes
- *               leaves the counters at zero again (after a call that raised
- *               PKV_FLAG_WAIT_TIMEOUT, zero it again).  Calls that share a
+ *               ZERO-FILLED before its first use (a new allocation at a
+ *               reused address counts as a first use); every call that
+ *               completes leaves the counters at zero again, and a call
+ *               whose counters reach further than the previous call's on the
+ *               same address (a larger batch) clears the difference on
+ *               `stream` first.  After a call that raised
+ *               PKV_FLAG_WAIT_TIMEOUT, zero it again.  Calls that share a
  *               workspace must not overlap in time.
  *   out         [batch][Hq][d] bf16 (written)
  *   out_lse     [batch][Hq] fp32 natural-log softmax denominators, or NULL

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "decode.cuh"
 #include "kv_append.cuh"
@@ -161,6 +162,27 @@ WorkspaceLayout workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t S) {
   w.part_o = w.part_lse + align256(static_cast<size_t>(B) * Hq * S * 4);
   w.total = w.part_o + align256(static_cast<size_t>(B) * Hq * S * D * 4);
   return w;
+}
+
+// Leading bytes of each workspace known to be zero when its last call ended
+// (the counters of that call's layout; calls that complete leave them zero).
+// A call whose counters reach further -- a larger batch moves the later
+// regions, whose old contents then sit where the new counters go -- first
+// clears the difference on its stream.  Keyed by workspace address; an
+// address seen for the first time is cleared over its whole counter region.
+std::unordered_map<const void*, size_t> g_ws_zero;
+constexpr size_t kMaxTrackedWorkspaces = 4096;
+
+int prepare_workspace(void* ws, size_t need, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  auto it = g_ws_zero.find(ws);
+  const size_t have = it == g_ws_zero.end() ? 0 : it->second;
+  if (need > have &&
+      cudaMemsetAsync(static_cast<uint8_t*>(ws) + have, 0, need - have, stream) != cudaSuccess)
+    return PKV_ERR_CUDA;
+  if (it == g_ws_zero.end() && g_ws_zero.size() >= kMaxTrackedWorkspaces) g_ws_zero.clear();
+  g_ws_zero[ws] = need;
+  return PKV_OK;
 }
 
 // ------------------------------------------------------------ decode launch
@@ -371,6 +393,7 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   prm.partition = partition_tokens;
   prm.scale_log2 = scale * 1.4426950408889634f;
   auto s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = prepare_workspace(workspace, wl.zero_bytes, s)) != PKV_OK) return st;
   if (D == 128) return dispatch_decode_group<128>(group, prm, dev.sm_count, s);
   return dispatch_decode_group<64>(group, prm, dev.sm_count, s);
 }

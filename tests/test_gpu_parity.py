@@ -166,6 +166,25 @@ def test_decode_reuses_workspace(pkv):
     check_no_flags(pkv)
 
 
+def test_decode_workspace_survives_batch_growth(pkv):
+    # a larger batch moves the workspace's later regions, so its counters land
+    # where a smaller batch left split counts and partials; the library must
+    # clear them before the larger call
+    small = make_workload("qwen3_decode", 21, B=5, len_lo=300, len_hi=3000)
+    big = make_workload("qwen3_decode", 22, B=12, len_lo=300, len_hi=3000)
+    max_kv = max(small.max_pages * small.page_size, big.max_pages * big.page_size)
+    ws = pkv.decode_workspace(big.B, big.num_q_heads, big.head_dim, max_kv, 0)
+    ds_small, ds_big = DeviceStep(pkv, small), DeviceStep(pkv, big)
+    ds_small.append()
+    ds_big.append()
+    ref = ds_big.decode(partition=0).clone()  # a fresh workspace of its own
+    for part in (0, 512, 0):
+        ds_small.decode(partition=part, workspace=ws)
+    got = ds_big.decode(partition=0, workspace=ws)
+    assert np.abs(bf16_to_f64(got) - bf16_to_f64(ref)).max() <= MAX_ABS
+    check_no_flags(pkv)
+
+
 # ------------------------------------------------------- split-K combine API
 @pytest.mark.parametrize("d", [64, 128])
 def test_split_k_combine(pkv, d):
