@@ -41,6 +41,21 @@ METRIC = "paged decode attention KV-read GB/s (% of 8 TB/s HBM); mixed-batch tok
 HEADLINE = "qwen3_decode"
 
 
+def profiled_traffic(key):
+    """DRAM bytes (read + write) per launch of a kernel, from the ncu capture
+    recorded in profiles/traffic.json -- or None when the kernel's source has
+    changed since that capture (its sha256 no longer matches)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[key]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    return rec["dram_bytes_per_launch"] if digest == rec["source_sha256"] else None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -427,7 +442,7 @@ def main():
                    "l2": "inputs larger than L2 (KV read per step > 126 MB), no flush"},
         "pct_of_8TBs": 100 * value / HBM_NOMINAL_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
+                     "frac": achieved / hbm, "traffic": profiled_traffic("decode_partition_qwen3_decode"),
                      "kernel": "decode split-K partition + combine (one pkv_paged_attn_decode call)",
                      "peak_source": f"{peak_src} hbm_gbs", "pct_of_8TBs": 100 * achieved / HBM_NOMINAL_GBS},
         "cpu_baseline": ({"value": cpu_rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
