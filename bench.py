@@ -241,24 +241,33 @@ def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    # timed region: K whole steps, nothing recorded between the kernels (an
+    # event between two launches would serialise them and cost the
+    # programmatic-dependent-launch overlap)
     t0, t1 = mk(), mk()
     with ClockSampler(clocks_index) as clk:
         t0.record()
         for i in range(steps):
-            g.step(g.dev, evs[i])
+            g.step(g.dev)
         t1.record()
         torch.cuda.synchronize()
     total_ms = t0.elapsed_time(t1)
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    # second timed pass of K steps with CUDA events around each attention call
+    # on its stream: the per-call kernel durations of the roofline
+    torch.cuda.synchronize()
+    for i in range(steps):
+        g.step(g.dev, evs[i])
+    torch.cuda.synchronize()
     per = {"pre": [], "dec": []}
     for i in range(steps):
         if g.pre:
             per["pre"].append(evs[i]["pre"][0].elapsed_time(evs[i]["pre"][1]))
         if g.dec:
             per["dec"].append(evs[i]["dec"][0].elapsed_time(evs[i]["dec"][1]))
-    if dist is not None:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
     # end-to-end through the public API with host buffers
     for _ in range(warmup):
         g.step_e2e()
@@ -444,6 +453,7 @@ def main():
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": profiled_traffic("decode_partition_qwen3_decode"),
                      "kernel": "decode split-K partition + combine (one pkv_paged_attn_decode call)",
+                     "timing": "CUDA events around each decode call over a second pass of the K timed steps",
                      "peak_source": f"{peak_src} hbm_gbs", "pct_of_8TBs": 100 * achieved / HBM_NOMINAL_GBS},
         "cpu_baseline": ({"value": cpu_rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
                           "sample": sample, "seconds": cpu_secs} if cpu_rate else None),

@@ -268,6 +268,9 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   const int log2P = 31 - __clz(p.P);  // P is a power of two
   static_assert((T == 8 || T == 16) && (D == 64 || D == 128), "head_dim 64 or 128");
   static_assert(NS >= 2, "at least two stages per warp");
+  // launched as a programmatic dependent: nothing global is read before the
+  // kernel ahead of it on the stream (usually the append) has completed
+  pdl_wait();
 
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -377,7 +380,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   __syncthreads();
   // let a dependent launch (the combine kernel) be scheduled now; it waits
   // for this whole grid to finish before reading anything
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_launch_dependents();
   const int part = misc[0], nF = misc[1], total = misc[1] + misc[2];
   // automatic split: warp w < Weff (= misc[0]) takes quanta
   // [floor(w*Q/Weff), floor((w+1)*Q/Weff)); the slice holding quantum x is
@@ -806,7 +809,7 @@ __global__ void __launch_bounds__(32 * kCombineMaxWarps) combine_kernel(
   const long long row = blockIdx.x;
   // launched as a programmatic dependent of the partition kernel: wait for
   // that grid to complete (a no-op when launched normally)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
   int n = num_splits[row / rows_per_entry];
   if (n <= skip_below) return;
   n = max(0, min(n, S_max));

@@ -20,6 +20,9 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict_
                                                         int32_t num_kv_heads, int32_t page_size,
                                                         int64_t num_slots) {
   constexpr int kChunks = D / 8;  // 16-byte chunks per row
+  // the attention kernel that usually follows may be scheduled now; it waits
+  // for this grid to complete before reading the pool
+  pdl_launch_dependents();
   const int64_t total = static_cast<int64_t>(T) * num_kv_heads * kChunks;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {

@@ -95,6 +95,26 @@ int check_heads(int32_t num_q_heads, const pkv_pool_desc& pool, int* group) {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
 
+// Launch as a programmatic dependent of the previous kernel on the stream:
+// the kernel starts early and waits (pdl_wait) before its first global read,
+// so its launch latency overlaps the tail of the kernel ahead of it.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+               Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) return PKV_ERR_CUDA;
+  return launch_status();
+}
+
 // warps per combine CTA: about one per eight splits, a power of two in [1, 8]
 int combine_warps(int32_t max_splits) {
   int w = 1;
@@ -215,8 +235,7 @@ int launch_decode(const pkv::decode::Params& prm, int sm_count, cudaStream_t str
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return PKV_ERR_CUDA;
-  kernel<<<sm_count, W * 32, smem, stream>>>(prm);
-  if (launch_status() != PKV_OK) return PKV_ERR_CUDA;
+  if (launch_pdl(kernel, dim3(sm_count), dim3(W * 32), smem, stream, prm) != PKV_OK) return PKV_ERR_CUDA;
   if (prm.partition < 0) return PKV_OK;  // every request is one split
   if (prm.partition == 0) {
     // automatic split: groups of at most kFusedMergeMax splits were merged in
@@ -264,8 +283,8 @@ int launch_prefill(const pkv::prefill::Params& prm, const CUtensorMap& qmap, con
   if (blocks > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
   pkv::prefill::Params args = prm;
   args.qtiles = static_cast<int32_t>(tiles);
-  kernel<<<static_cast<unsigned>(blocks), pkv::prefill::kThreads, smem, stream>>>(qmap, kmap, vmap, args);
-  return launch_status();
+  return launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(pkv::prefill::kThreads), smem, stream, qmap,
+                    kmap, vmap, args);
 }
 
 template <int D>

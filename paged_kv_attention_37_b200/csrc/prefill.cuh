@@ -77,6 +77,10 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
   constexpr int QPOS = kM / G;  // chunk positions per tile
   constexpr uint32_t kIdescS = idesc_bf16_f32(kM, kN, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, D, false, true);
+  // launched as a programmatic dependent (see pdl_wait): nothing global is
+  // read before the kernel ahead of it has completed
+  pdl_wait();
+  pdl_launch_dependents();
 
   // ---- which tile.  Order 1: the query tiles of one (request, KV head) are
   // adjacent, heaviest (last) first, so the CTAs that read the same keys run

@@ -22,6 +22,18 @@ __device__ __forceinline__ void raise_flag(uint32_t bits) { atomicOr(&g_error_fl
 // gives up so the context stays usable.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is still
+// running; pdl_wait() blocks until that kernel has completed and its writes
+// are visible (a no-op for a normal launch), so it must come before the first
+// read of anything an earlier kernel may have written.  pdl_launch_dependents()
+// lets the next such kernel be scheduled once every CTA of this grid has
+// signalled or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
