@@ -230,6 +230,30 @@ def prefill_flops(w):
     return tot
 
 
+def max_over_ranks(dist, x, device="cuda"):
+    """The largest of every rank's x (the timing rule for N replicas): an
+    all-reduce MAX over the process group, or x itself without one."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(world, bytes_per_rank, ms):
+    """Whole-job GB/s of `world` replicas that each move bytes_per_rank in ms."""
+    return world * bytes_per_rank / (ms / 1e3) / 1e9
+
+
+def emit(rank, line):
+    """Print the JSON line on rank 0 only; True when printed."""
+    if rank != 0:
+        return False
+    print(json.dumps(line))
+    return True
+
+
 def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
     w = make_workload(name, 0)
     g = GpuWorkload(pkv, torch, w)
@@ -251,11 +275,7 @@ def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
             g.step(g.dev)
         t1.record()
         torch.cuda.synchronize()
-    total_ms = t0.elapsed_time(t1)
-    if dist is not None:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(dist, t0.elapsed_time(t1))
     # second timed pass of K steps with CUDA events around each attention call
     # on its stream: the per-call kernel durations of the roofline
     torch.cuda.synchronize()
@@ -278,11 +298,7 @@ def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
         g.step_e2e()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1))
     flags = pkv.pkv_device_error_flags(clear=True)
     if flags:
         raise RuntimeError(f"device error flags {flags:#x} during {name}")
@@ -349,7 +365,8 @@ def cpu_oracle_rate(name, budget_s=12.0):
 
 
 def reference_arm(args):
-    """The CPU oracle as the reference arm (rank 0 only)."""
+    """The CPU oracle as the reference arm: rank 0 alone runs it; the other
+    ranks of a torchrun launch exit 0 without work."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
@@ -371,7 +388,7 @@ def reference_arm(args):
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line))
+    emit(rank, line)
     return 0
 
 
@@ -431,9 +448,9 @@ def main():
 
     w = head["w"]
     kv_bytes = head["kv_bytes_dec"]
-    value = world * kv_bytes / (head["ms_per_step"] / 1e3) / 1e9
-    achieved = kv_bytes / (head["dec_ms"] / 1e3) / 1e9
-    e2e_value = world * kv_bytes / (head["e2e_ms_per_step"] / 1e3) / 1e9
+    value = aggregate_gbs(world, kv_bytes, head["ms_per_step"])
+    achieved = aggregate_gbs(1, kv_bytes, head["dec_ms"])
+    e2e_value = aggregate_gbs(world, kv_bytes, head["e2e_ms_per_step"])
     if rank != 0:
         if dist is not None:
             dist.barrier()
@@ -463,7 +480,7 @@ def main():
         "clocks": head["clocks"],
         "workloads": extra,
     }
-    print(json.dumps(line))
+    emit(rank, line)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
