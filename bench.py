@@ -118,6 +118,25 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- GPU side
+class Packed:
+    """Tensors of the given (dtype, shape) as views into one byte buffer, each
+    at a 256-byte aligned offset; pinned when on the host."""
+
+    def __init__(self, torch, specs, device):
+        offs, n = {}, 0
+        for k, (dt, shape) in specs.items():
+            offs[k] = n
+            nb = int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+            n += (nb + 255) // 256 * 256
+        self.buf = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+        if device == "cpu":
+            self.buf = self.buf.pin_memory()
+        self.views = {}
+        for k, (dt, shape) in specs.items():
+            nb = int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+            self.views[k] = self.buf[offs[k]:offs[k] + nb].view(dt).view(shape)
+
+
 class GpuWorkload:
     """Device buffers for one workload: pools with every request's context
     (drawn on the GPU, seeded), and the step's inputs (host-generated)."""
@@ -159,18 +178,38 @@ class GpuWorkload:
                 "ctx_pre": torch.from_numpy(np.ascontiguousarray(w.ctx_lens[pre])),
                 "pt_pre": torch.from_numpy(np.ascontiguousarray(w.page_table[pre])),
             })
-        self.host = {k: t.pin_memory() for k, t in self.host.items()}
-        self.dev = {k: t.to(dev) for k, t in self.host.items()}
+        # every step input lives in one pinned host buffer and in each of two
+        # device buffers (views at 256-byte aligned offsets): the end-to-end
+        # leg moves a step's inputs with a single copy, double-buffered
+        specs = {k: (t.dtype, tuple(t.shape)) for k, t in self.host.items()}
+        hin = Packed(torch, specs, "cpu")
+        for k, t in self.host.items():
+            hin.views[k].copy_(t)
+        self.in_host = hin
+        self.in_dev = [Packed(torch, specs, dev) for _ in range(2)]
+        for d in self.in_dev:
+            d.buf.copy_(hin.buf)
+        self.host = hin.views
+        self.dev = self.in_dev[0].views
+        self.dev_sets = [d.views for d in self.in_dev]
         self.dec, self.pre = dec, pre
         self.max_q = int(w.new_lens[pre].max()) if pre else 0
         if dec:
             self.ws = pkv.decode_workspace(len(dec), w.num_q_heads, w.head_dim,
                                            w.max_pages * w.page_size, 0)
-            self.out_dec = torch.empty_like(self.dev["q_dec"])
-            self.out_dec_host = torch.empty_like(self.out_dec, device="cpu").pin_memory()
+        # outputs: one packed device buffer per set, read back with one copy
+        ospecs = {}
+        if dec:
+            ospecs["dec"] = (torch.bfloat16, tuple(self.dev["q_dec"].shape))
         if pre:
-            self.out_pre = torch.empty_like(self.dev["q_pre"])
-            self.out_pre_host = torch.empty_like(self.out_pre, device="cpu").pin_memory()
+            ospecs["pre"] = (torch.bfloat16, tuple(self.dev["q_pre"].shape))
+        self.out_dev = [Packed(torch, ospecs, dev) for _ in range(2)]
+        self.out_host = [Packed(torch, ospecs, "cpu") for _ in range(2)]
+        self.out_sets = [d.views for d in self.out_dev]
+        if dec:
+            self.out_dec = self.out_sets[0]["dec"]
+        if pre:
+            self.out_pre = self.out_sets[0]["pre"]
         torch.cuda.synchronize()
 
     def bits(self, a):
@@ -182,42 +221,64 @@ class GpuWorkload:
     def launches_per_step(self):
         return 1 + (2 if self.dec else 0) + (1 if self.pre else 0)
 
-    def step(self, d, ev=None):
+    def step(self, d, ev=None, outs=None):
         """One pass of the hot path on device buffers d; ev optionally brackets
-        the prefill and decode calls with CUDA events."""
+        the prefill and decode calls with CUDA events; outs picks the output
+        buffers (default: the first set)."""
         pkv, w = self.pkv, self.w
+        out_pre = outs["pre"] if outs is not None and self.pre else getattr(self, "out_pre", None)
+        out_dec = outs["dec"] if outs is not None and self.dec else getattr(self, "out_dec", None)
         pkv.pkv_kv_append(d["k_new"], d["v_new"], d["slots"], self.k_pool, self.v_pool)
         if self.pre:
             if ev is not None:
                 ev["pre"][0].record()
             pkv.pkv_paged_attn_chunked_prefill(d["q_pre"], d["cu_q"], d["ctx_pre"], self.k_pool,
                                                self.v_pool, d["pt_pre"], w.scale, self.max_q,
-                                               out=self.out_pre)
+                                               out=out_pre)
             if ev is not None:
                 ev["pre"][1].record()
         if self.dec:
             if ev is not None:
                 ev["dec"][0].record()
             pkv.pkv_paged_attn_decode(d["q_dec"], self.k_pool, self.v_pool, d["pt_dec"],
-                                      d["len_dec"], w.scale, 0, workspace=self.ws, out=self.out_dec)
+                                      d["len_dec"], w.scale, 0, workspace=self.ws, out=out_dec)
             if ev is not None:
                 ev["dec"][1].record()
 
-    def step_e2e(self):
-        """Same step through the public API from pinned host buffers: H2D of the
-        step's inputs, the kernels, D2H of the outputs."""
-        for k, t in self.host.items():
-            self.dev[k].copy_(t, non_blocking=True)
-        self.step(self.dev)
-        if self.dec:
-            self.out_dec_host.copy_(self.out_dec, non_blocking=True)
-        if self.pre:
-            self.out_pre_host.copy_(self.out_pre, non_blocking=True)
+    def run_e2e(self, steps):
+        """`steps` steps through the public API from pinned host buffers: every
+        step copies its inputs host-to-device, runs the kernels and reads its
+        outputs back.  Two buffer sets and a copy stream let the copies of one
+        step overlap the kernels of its neighbours; the caller times the whole
+        run on the current stream (it waits for the copy stream at the end)."""
+        torch = self.torch
+        main = torch.cuda.current_stream()
+        cs = self._copy_stream = getattr(self, "_copy_stream", None) or torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        cs.wait_stream(main)
+        for i in range(steps):
+            b = i & 1
+            with torch.cuda.stream(cs):
+                if i >= 2:
+                    cs.wait_event(ev_done[b])  # the kernels of step i-2 no longer read set b
+                self.in_dev[b].buf.copy_(self.in_host.buf, non_blocking=True)
+                ev_in[b].record(cs)
+            main.wait_event(ev_in[b])
+            if i >= 2:
+                main.wait_event(ev_out[b])  # step i-2's outputs have left set b
+            self.step(self.dev_sets[b], outs=self.out_sets[b])
+            ev_done[b].record(main)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev_done[b])
+                self.out_host[b].buf.copy_(self.out_dev[b].buf, non_blocking=True)
+                ev_out[b].record(cs)
+        main.wait_stream(cs)
 
     def io_bytes(self):
-        h2d = sum(t.numel() * t.element_size() for t in self.host.values())
-        d2h = (self.out_dec.numel() * 2 if self.dec else 0) + (self.out_pre.numel() * 2 if self.pre else 0)
-        return h2d, d2h
+        """Bytes copied per end-to-end step (packed buffers, alignment included)."""
+        return self.in_host.buf.numel(), self.out_dev[0].buf.numel()
 
 
 def prefill_flops(w):
@@ -289,13 +350,11 @@ def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
         if g.dec:
             per["dec"].append(evs[i]["dec"][0].elapsed_time(evs[i]["dec"][1]))
     # end-to-end through the public API with host buffers
-    for _ in range(warmup):
-        g.step_e2e()
+    g.run_e2e(warmup)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(steps):
-        g.step_e2e()
+    g.run_e2e(steps)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1))
