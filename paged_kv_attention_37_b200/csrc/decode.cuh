@@ -456,6 +456,15 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     pid_cur = lane < it_npg ? __ldg(ptab + lane) : -1;
     pid_next = 32 + lane < it_npg ? __ldg(ptab + 32 + lane) : -1;
     active = true;
+    if (balanced && bq < bq_end && lane == 0) {
+      // the next item of the slice is known: pull its first page-table line
+      // into L1 now, so starting it does not wait on the page table
+      const int r2 = upper_index(prefF, p.B, bq);
+      const int gq2 = (prefF[r2 + 1] - prefF[r2]) / p.Hkv;
+      const int g2 = (bq - prefF[r2]) / gq2;
+      const int t2 = (bq - prefF[r2] - g2 * gq2) * kPartitionQuantum;
+      prefetch_l1(p.page_table + static_cast<size_t>(r2) * p.max_pages + (t2 >> log2P));
+    }
   };
 
   // Issue the next chunk of the current (or next) item into stage n % NS.
@@ -752,11 +761,12 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
         const size_t gi = static_cast<size_t>(it.r) * p.Hkv + it.g;
         if (it.s == 0 && lane == 0) p.group_splits[gi] = it.nsplit;
         if (it.nsplit <= kFusedMergeMax) {
-          // the warp that finishes the group's last split merges the partials
-          __threadfence();
+          // the warp that finishes the group's last split merges the partials;
+          // lane 0's release add publishes every lane's partial stores (they
+          // precede it through the warp barrier)
           __syncwarp();
           uint32_t done = 0;
-          if (lane == 0) done = atomicAdd(p.group_done + gi, 1u);
+          if (lane == 0) done = atomic_add_release_gpu(p.group_done + gi, 1u);
           done = __shfl_sync(0xffffffffu, done, 0);
           if (done == static_cast<uint32_t>(it.nsplit - 1)) {
             __threadfence();

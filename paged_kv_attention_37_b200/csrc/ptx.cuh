@@ -34,6 +34,20 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Fire-and-forget prefetch of the line holding `ptr` into L1.
+__device__ __forceinline__ void prefetch_l1(const void* ptr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));
+}
+
+// atomicAdd with release semantics at GPU scope: memory operations that
+// precede it (in this thread, or in threads it has synchronised with) are
+// visible to any thread that observes the add and then acquires.
+__device__ __forceinline__ uint32_t atomic_add_release_gpu(uint32_t* ptr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
