@@ -53,7 +53,9 @@
 namespace pkv {
 namespace decode {
 
-constexpr int kBoxRows = 16;     // token rows per copy unit (a page, or half of one)
+#ifndef PKV_DECODE_CHUNK_BYTES
+#define PKV_DECODE_CHUNK_BYTES 8192
+#endif
 #ifndef PKV_DECODE_CPASYNC
 #define PKV_DECODE_CPASYNC 1
 #endif
@@ -63,8 +65,14 @@ constexpr int kBoxRows = 16;     // token rows per copy unit (a page, or half of
 constexpr bool kCpAsync = PKV_DECODE_CPASYNC != 0;
 template <int D>
 struct Chunk {
-  static constexpr int kTokens = 2048 / D;             // tokens per pipeline stage (8 KB of K+V)
-  static constexpr int kBoxes = kTokens / kBoxRows;    // 16-row pieces per stage (per K or V)
+  // tokens per pipeline stage: PKV_DECODE_CHUNK_BYTES of K+V (16 at d=128
+  // and 8 KB)
+  static constexpr int kTokens = PKV_DECODE_CHUNK_BYTES / (4 * D);
+  // token rows per copy unit: one page of 16, half of a 32-token page, or a
+  // part of either; each unit is one contiguous run of the pool
+  static constexpr int kBoxRows = kTokens < 16 ? kTokens : 16;
+  static constexpr int kBoxes = kTokens / kBoxRows;    // copy units per stage (per K or V)
+  static_assert(kTokens >= 8 && 32 % kTokens == 0, "chunks tile a 32-token quantum");
 };
 constexpr int kItemSlots = 8;    // per-warp ring of item descriptors
 // Automatic split (partition_tokens == 0): the padded token-heads of the
@@ -478,7 +486,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     const int tok0 = it_k * kTok;  // relative to the item's first token (a page start)
     const int ntok = it_nch == 0 ? 0 : min(kTok, it_ntok - tok0);
     const int flags = (it_k == 0 ? kFirst : 0) | (it_k + 1 >= it_nch ? kLast : 0);
-    const int nbox = (ntok + kBoxRows - 1) / kBoxRows;
+    const int nbox = (ntok + CK::kBoxRows - 1) / CK::kBoxRows;
     // each 16-row piece lies inside one page: page-table entry (tok >> log2P),
     // first row (tok & (P-1)); out-of-range page ids read page 0 instead
     // (wrong values, no stray access) and raise PKV_FLAG_BAD_PAGE
@@ -487,7 +495,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     for (int b = 0; b < CK::kBoxes; ++b) {
       rows[b] = 0;
       if (b < nbox) {
-        const int pi = (tok0 + b * kBoxRows) >> log2P;
+        const int pi = (tok0 + b * CK::kBoxRows) >> log2P;
         while (pi >= pid_base + 32) {
           pid_base += 32;
           pid_cur = pid_next;
@@ -498,7 +506,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
           if (lane == 0) raise_flag(PKV_FLAG_BAD_PAGE);
           page = 0;
         }
-        rows[b] = (static_cast<size_t>(page) * p.Hkv + it_g) * p.P + ((tok0 + b * kBoxRows) & (p.P - 1));
+        rows[b] = (static_cast<size_t>(page) * p.Hkv + it_g) * p.P + ((tok0 + b * CK::kBoxRows) & (p.P - 1));
       }
     }
     const uint32_t st = wbase + stage * LY::kStageBytes;
@@ -507,7 +515,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     if (lane == 0) fifo[stage] = ChunkInfo{it_slot, ntok, flags, it_qslot};
     if constexpr (kCpAsync) {
       if (ntok > 0) {
-        constexpr int kPieces = kBoxRows * D / 8;  // 16-byte pieces per 16-row piece
+        constexpr int kPieces = CK::kBoxRows * D / 8;  // 16-byte pieces per 16-row piece
 #pragma unroll
         for (int b = 0; b < CK::kBoxes; ++b) {
           if (b >= nbox) break;
@@ -515,8 +523,8 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
           const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + rows[b] * D);
 #pragma unroll
           for (int i = lane; i < kPieces; i += 32) {
-            cp_async16(st + b * (kBoxRows * D * 2) + i * 16, ksrc + i * 16);
-            cp_async16(st + LY::kKBytes + b * (kBoxRows * D * 2) + i * 16, vsrc + i * 16);
+            cp_async16(st + b * (CK::kBoxRows * D * 2) + i * 16, ksrc + i * 16);
+            cp_async16(st + LY::kKBytes + b * (CK::kBoxRows * D * 2) + i * 16, vsrc + i * 16);
           }
         }
         if (it_k == 0) {
@@ -528,14 +536,14 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     } else if (lane == 0) {
       if (ntok > 0) {
         const bool with_q = it_k == 0;
-        const uint32_t bytes = static_cast<uint32_t>(nbox * kBoxRows * D * 2 * 2) +
+        const uint32_t bytes = static_cast<uint32_t>(nbox * CK::kBoxRows * D * 2 * 2) +
                                (with_q ? static_cast<uint32_t>(G * D * 2) : 0u);
         mbar_arrive_expect_tx(full_bar(stage), bytes);
 #pragma unroll
         for (int b = 0; b < CK::kBoxes; ++b) {
           if (b >= nbox) break;
-          bulk_load(st + b * (kBoxRows * D * 2), p.k_pool + rows[b] * D, kBoxRows * D * 2, full_bar(stage));
-          bulk_load(st + LY::kKBytes + b * (kBoxRows * D * 2), p.v_pool + rows[b] * D, kBoxRows * D * 2,
+          bulk_load(st + b * (CK::kBoxRows * D * 2), p.k_pool + rows[b] * D, CK::kBoxRows * D * 2, full_bar(stage));
+          bulk_load(st + LY::kKBytes + b * (CK::kBoxRows * D * 2), p.v_pool + rows[b] * D, CK::kBoxRows * D * 2,
                     full_bar(stage));
         }
         if (with_q) bulk_load(qdst, qsrc, G * D * 2, full_bar(stage));
