@@ -13,10 +13,11 @@
 // produces the outputs of all G query heads of the group, so every K/V byte
 // is read from HBM once and used G times.  Two schedules:
 //   automatic split (partition_tokens == 0): each group is padded to whole
-//   32-token quanta and the groups are laid end to end; warp w takes the
+//   32-token quanta, led by kGroupCost empty quanta that stand for its fixed
+//   per-piece cost, and the groups are laid end to end; warp w takes the
 //   w-th of Weff equal slices (to one quantum; at least kMinShare tokens) of
-//   that line, so every warp streams the same number of bytes and all finish
-//   together.  A slice may
+//   that line, so every warp has the same work and all finish together.
+//   A slice may
 //   end inside a group and the next one continue it: such a group's pieces
 //   are split-K partials, merged by the warp that finishes the group's last
 //   piece (at most kFusedMergeMax pieces) or by combine_kernel (more).
@@ -81,6 +82,14 @@ constexpr int kItemSlots = 8;    // per-warp ring of item descriptors
 constexpr int kMinShare = 128;
 
 constexpr int kPartitionQuantum = 32;  // split lengths are multiples of this
+// Each group enters the balanced slicing with this many extra quanta ahead of
+// its tokens, which hold no tokens: they stand for the fixed cost of starting
+// and ending a piece of a group (page-table fetch, output or partial write,
+// and the merge that the warp holding a group's first piece usually does).
+#ifndef PKV_DECODE_GROUP_COST
+#define PKV_DECODE_GROUP_COST 2
+#endif
+constexpr int kGroupCost = PKV_DECODE_GROUP_COST;
 // A (request, KV head) group cut into at most this many splits is merged
 // inside the partition kernel by the warp that finishes its last split;
 // groups with more splits are merged by combine_kernel, whose CTAs spread the
@@ -303,7 +312,8 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
 
   // ---- plan (warp 0).  Automatic split: every (request, KV head) group is
   // padded to whole 32-token quanta (an empty request to one, so its zero
-  // output is written); prefF[r] is the first quantum of request r's groups
+  // output is written) plus kGroupCost empty leading quanta; prefF[r] is the
+  // first quantum of request r's groups
   // in the concatenation, and warp w takes quanta [w*share, (w+1)*share).
   // Fixed partition: whole-partition items first (prefF), then one remainder
   // item per (request, KV head) whose length is not a multiple of the
@@ -333,7 +343,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       for (int base = 0; base < p.B; base += 32) {
         const int r = base + lane;
         int nq = 0;
-        if (r < p.B) nq = max(1, (lens[r] + kPartitionQuantum - 1) / kPartitionQuantum) * p.Hkv;
+        if (r < p.B) nq = (max(1, (lens[r] + kPartitionQuantum - 1) / kPartitionQuantum) + kGroupCost) * p.Hkv;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int y = __shfl_up_sync(0xffffffffu, nq, o);
@@ -408,20 +418,29 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   auto fetch = [&]() {
     int r, g, s, t0, ntok, nsplit;
     if (balanced) {
-      // next piece of this warp's slice: the rest of the group at bq
-      if (bq >= bq_end) {
-        more = false;
-        return;
+      // next piece of this warp's slice: the rest of the group at bq; a
+      // piece that holds only a group's cost quanta is no item
+      int first, iend;
+      for (;;) {
+        if (bq >= bq_end) {
+          more = false;
+          return;
+        }
+        r = upper_index(prefF, p.B, bq);
+        const int gq = (prefF[r + 1] - prefF[r]) / p.Hkv;  // quanta per group of request r
+        g = (bq - prefF[r]) / gq;
+        const int gstart = prefF[r] + g * gq;
+        first = gstart + kGroupCost;  // the group's first token quantum
+        iend = min(gstart + gq, bq_end);
+        if (iend > first) {
+          nsplit = slice_of(gstart + gq - 1) - slice_of(first) + 1;
+          break;
+        }
+        bq = iend;
       }
-      r = upper_index(prefF, p.B, bq);
-      const int gq = (prefF[r + 1] - prefF[r]) / p.Hkv;  // quanta per group of request r
-      g = (bq - prefF[r]) / gq;
-      const int gstart = prefF[r] + g * gq, gend = gstart + gq;
-      const int iend = min(gend, bq_end);
-      t0 = (bq - gstart) * kPartitionQuantum;
-      ntok = max(0, min((iend - gstart) * kPartitionQuantum, lens[r]) - t0);
-      s = wid - slice_of(gstart);
-      nsplit = slice_of(gend - 1) - slice_of(gstart) + 1;
+      t0 = (max(bq, first) - first) * kPartitionQuantum;
+      ntok = max(0, min((iend - first) * kPartitionQuantum, lens[r]) - t0);
+      s = wid - slice_of(first);
       bq = iend;
     } else {
     int idx = 0;
@@ -470,7 +489,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       const int r2 = upper_index(prefF, p.B, bq);
       const int gq2 = (prefF[r2 + 1] - prefF[r2]) / p.Hkv;
       const int g2 = (bq - prefF[r2]) / gq2;
-      const int t2 = (bq - prefF[r2] - g2 * gq2) * kPartitionQuantum;
+      const int t2 = max(0, bq - prefF[r2] - g2 * gq2 - kGroupCost) * kPartitionQuantum;
       prefetch_l1(p.page_table + static_cast<size_t>(r2) * p.max_pages + (t2 >> log2P));
     }
   };
