@@ -145,8 +145,8 @@ PKV_API size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, in
  *               slices is merged from partials); -1 = never split; otherwise
  *               a multiple of 32 in [32, 65536]
  *   workspace   device scratch of pkv_decode_workspace_bytes(...) bytes,
- *               holding split partials, two scheduling counters and one
- *               finished-split counter per (request, KV head).  It must be
+ *               holding split partials, two scheduling counters and the
+ *               merge-tree counters of each (request, KV head).  It must be
  *               ZERO-FILLED before its first use (a new allocation at a
  *               reused address counts as a first use); every call that
  *               completes leaves the counters at zero again, and a call
@@ -159,10 +159,11 @@ PKV_API size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, in
  *   out_lse     [batch][Hq] fp32 natural-log softmax denominators, or NULL
  *
  * Requests that are not split are written by the partition kernel directly.
- * Split ones go through fp32 partials: with the automatic split, a (request,
- * KV head) cut into at most 8 pieces is merged inside the partition kernel by
- * the warp finishing its last piece, longer ones (and every split request of
- * a fixed partition) by a second, combine kernel.
+ * Split ones go through fp32 partials.  With the automatic split, the pieces
+ * of a (request, KV head) are merged inside the partition kernel by a tree of
+ * merges of at most 8 partials each, every node merged by the warp that
+ * finishes its last child, so one kernel does the whole call.  With a fixed
+ * partition, a second, combine kernel merges the split requests.
  */
 PKV_API int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads,
                           const void* k_pool, const void* v_pool, pkv_pool_desc pool,

@@ -19,8 +19,9 @@
 //   that line, so every warp has the same work and all finish together.
 //   A slice may
 //   end inside a group and the next one continue it: such a group's pieces
-//   are split-K partials, merged by the warp that finishes the group's last
-//   piece (at most kFusedMergeMax pieces) or by combine_kernel (more).
+//   are split-K partials, merged inside the kernel by a tree of merges of
+//   at most kMergeFanIn partials, each done by the warp that completes the
+//   node's last child.
 //   fixed partition: items are (r, g, split s) of the given length; whole
 //   partitions are handed out first and the shorter remainders last, from an
 //   atomic counter in the workspace (dynamic balancing over ragged lengths),
@@ -76,6 +77,10 @@ struct Chunk {
   static_assert(kTokens >= 8 && 32 % kTokens == 0, "chunks tile a 32-token quantum");
 };
 constexpr int kItemSlots = 8;    // per-warp ring of item descriptors
+// Merge-tree nodes above the first level whose first-level child this warp
+// completed, climbed after the warp's slice (a slice holds at most two
+// pieces of split groups: its first and its last).
+constexpr int kClimbSlots = 2;
 // Automatic split (partition_tokens == 0): the padded token-heads of the
 // batch are cut into one equal slice per warp, at least kMinShare tokens, so
 // every warp streams the same number of bytes and all finish together.
@@ -90,11 +95,35 @@ constexpr int kPartitionQuantum = 32;  // split lengths are multiples of this
 #define PKV_DECODE_GROUP_COST 2
 #endif
 constexpr int kGroupCost = PKV_DECODE_GROUP_COST;
-// A (request, KV head) group cut into at most this many splits is merged
-// inside the partition kernel by the warp that finishes its last split;
-// groups with more splits are merged by combine_kernel, whose CTAs spread the
-// partial reads over many SMs.
-constexpr int kFusedMergeMax = 8;
+// Automatic split: the pieces of a (request, KV head) group are merged inside
+// the partition kernel by a tree whose nodes merge at most kMergeFanIn
+// partials.  Level 0 holds the n pieces; level k+1 has ceil(n_k / fan-in)
+// nodes, node j merging children [j*fan-in, (j+1)*fan-in) of level k; the
+// single top node writes the output.  The warp whose increment completes a
+// node's child count merges it, so no warp waits and no second kernel runs.
+// Partial slots of a row: the pieces, then each inner level below the top.
+// The fan-in keeps one head's children at 4 KB (8 partials of 128 fp32 or
+// 16 of 64), so four heads' fit a warp's two 8 KB stage buffers at once.
+template <int D>
+constexpr int kMergeFanIn = D == 64 ? 16 : 8;
+
+__host__ __device__ constexpr int merge_tree_slots(int n, int fan_in) {
+  int total = n;
+  while (n > fan_in) {
+    n = (n + fan_in - 1) / fan_in;
+    total += n;
+  }
+  return total;
+}
+// merge nodes of that tree (the top one included): one counter each
+__host__ __device__ constexpr int merge_tree_nodes(int n, int fan_in) {
+  int total = 0;
+  while (n > 1) {
+    n = (n + fan_in - 1) / fan_in;
+    total += n;
+  }
+  return total;
+}
 constexpr float kLazyRescale = 8.0f;  // log2 units: move the running max when it grows > 2^8
 constexpr int kFirst = 1;  // first chunk of an item
 constexpr int kLast = 2;   // last chunk of an item
@@ -111,9 +140,8 @@ struct Params {
   float* part_lse;            // [B][Hq][S_max]
   int32_t* num_splits;        // [B]
   uint32_t* counters;         // [0] next item, [1] finished warps
-  uint32_t* group_done;       // [B*Hkv] splits finished per (request, KV head) (automatic split)
-  int32_t* group_splits;      // [B*Hkv] splits of each (request, KV head) (automatic split)
-  int32_t B, Hq, Hkv, P, max_pages, num_pages, S_max, partition;
+  uint32_t* group_done;       // [B*Hkv][merge_nodes] finished children per merge node (automatic split)
+  int32_t B, Hq, Hkv, P, max_pages, num_pages, S_max, partition, merge_nodes;
   float scale_log2;           // softmax scale * log2(e)
 };
 
@@ -137,7 +165,8 @@ struct Layout {
   static constexpr int kBarOff = kPbOff + kTok * G * 8;         // NS mbarriers
   static constexpr int kFifoOff = kBarOff + NS * 8;             // NS ChunkInfo
   static constexpr int kItemOff = kFifoOff + NS * 16;           // kItemSlots ItemInfo
-  static constexpr int kWarpBytes = (kItemOff + kItemSlots * 16 + 127) / 128 * 128;
+  static constexpr int kClimbOff = kItemOff + kItemSlots * 16;  // kClimbSlots ItemInfo
+  static constexpr int kWarpBytes = (kClimbOff + kClimbSlots * 16 + 127) / 128 * 128;
   // after the W warp blocks: misc[4], lens[B], prefF[B+1], prefR[B+1]
   static size_t plan_bytes(int B) { return 16 + (3 * static_cast<size_t>(B) + 2) * 4; }
   static size_t bytes(int W, int B) { return static_cast<size_t>(W) * kWarpBytes + plan_bytes(B) + 128; }
@@ -205,14 +234,95 @@ __device__ __forceinline__ float reduce_scatter_heads(float (&v)[G]) {
   return v[0];
 }
 
-// Merge the nsplit partials of the G query heads of one (request, KV head)
-// group: o = sum_s w_s o_s / sum_s w_s with w_s = exp(lse_s - max lse) (the
-// split-K rule of combine_kernel).  One warp; lane l owns output elements
-// [l*D/32, (l+1)*D/32).  Partials are read through L2 (other warps wrote them
-// during this launch), all splits of a head in one batch of loads, so a merge
-// costs about one memory round trip per head.  nsplit <= kFusedMergeMax.
+// Merge partial slots [base, base + cnt) of the G query heads of one
+// (request, KV head) group: o = sum_s w_s o_s / sum_s w_s with
+// w_s = exp(lse_s - max lse) (the split-K rule of combine_kernel), into the
+// bf16 output (kToOut) or into partial slot dst (normalised o and its lse,
+// for the next level of the tree).  One warp, after its slice: the partials
+// (other warps wrote them during this launch) are copied through L2 into the
+// warp's idle stage buffers, as many heads' at once as fit, so a merge costs
+// one memory round trip per batch of heads; lane l then owns elements
+// [l*D/32, (l+1)*D/32).  cnt <= kMergeFanIn<D>.
+template <int D, int G, int NS, bool kToOut>
+__device__ __forceinline__ void merge_staged(const Params& p, int r, int g, int base, int cnt, int dst, int lane,
+                                             uint32_t sbase, const float* sbuf) {
+  constexpr int FI = kMergeFanIn<D>;
+  constexpr int DPL = D / 32;
+  constexpr int kPieces = D * 4 / 16;  // 16-byte pieces of one partial row: 32 or 16
+  constexpr int kRows = 32 / kPieces;  // rows one warp-wide copy covers
+  constexpr int kFit = NS * Layout<D, G, NS>::kStageBytes / (FI * D * 4);
+  static_assert(kFit >= 1, "one head's partials fit the stage buffers");
+  constexpr int HB = kFit < G ? kFit : G;  // heads per batch
+  constexpr float kLog2e = 1.4426950408889634f;
+  const size_t row0 = static_cast<size_t>(r) * p.Hq + static_cast<size_t>(g) * G;
+  float ls[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+    ls[h] = lane < cnt ? __ldcg(p.part_lse + (row0 + h) * p.S_max + base + lane) : -INFINITY;
+#pragma unroll
+  for (int h0 = 0; h0 < G; h0 += HB) {
+    const int c = lane % kPieces;
+#pragma unroll
+    for (int hb = 0; hb < HB; ++hb) {
+      const float* src = p.part_o + ((row0 + h0 + hb) * p.S_max + base) * D + c * 4;
+      for (int sp = lane / kPieces; sp < cnt; sp += kRows)
+        cp_async16(sbase + static_cast<uint32_t>(((hb * FI + sp) * D + c * 4) * 4), src + static_cast<size_t>(sp) * D);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
+#pragma unroll
+    for (int hb = 0; hb < HB; ++hb) {
+      const int h = h0 + hb;
+      const float lh = ls[h];
+      const float M = warp_max(lh);
+      const float w = M == -INFINITY ? 0.f : fast_exp2((lh - M) * kLog2e);
+      const float den = warp_sum(w);
+      float acc[DPL];
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < FI; ++sp) {
+        const float ws = __shfl_sync(0xffffffffu, w, sp);
+        if (sp < cnt) {
+          const float* x = sbuf + (hb * FI + sp) * D + lane * DPL;
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(ws, x[e], acc[e]);
+        }
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      const float lse = den > 0.f ? M + logf(den) : -INFINITY;
+      if constexpr (kToOut) {
+        uint16_t* o = p.out + (row0 + h) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          *reinterpret_cast<uint2*>(o) =
+              make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+        } else {
+          *reinterpret_cast<uint32_t*>(o) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        }
+        if (p.out_lse != nullptr && lane == 0) p.out_lse[row0 + h] = lse;
+      } else {
+        const size_t prow = (row0 + h) * p.S_max + dst;
+        float* o = p.part_o + prow * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          *reinterpret_cast<float4*>(o) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        } else {
+          *reinterpret_cast<float2*>(o) = make_float2(acc[0] * inv, acc[1] * inv);
+        }
+        if (lane == 0) p.part_lse[prow] = lse;
+      }
+    }
+    __syncwarp();  // the next batch overwrites the stage buffers
+  }
+}
+
+// The same merge of a group's nsplit <= kMergeFanIn<D> pieces (slots
+// [0, nsplit)) into the output, inside the streaming loop, where the stage
+// buffers are busy: the partials come through registers, one head's batch of
+// loads at a time (more heads per batch spill the loop's registers), so it
+// costs about one memory round trip per head.
 template <int D, int G>
-__device__ __forceinline__ void merge_group(const Params& p, int r, int g, int nsplit, int lane) {
+__device__ __forceinline__ void merge_regs(const Params& p, int r, int g, int nsplit, int lane) {
   constexpr int DPL = D / 32;
   constexpr int HB = 1;  // heads per batch of loads
   constexpr float kLog2e = 1.4426950408889634f;
@@ -223,12 +333,12 @@ __device__ __forceinline__ void merge_group(const Params& p, int r, int g, int n
     ls[h] = lane < nsplit ? __ldcg(p.part_lse + (row0 + h) * p.S_max + lane) : -INFINITY;
 #pragma unroll
   for (int h0 = 0; h0 < G; h0 += HB) {
-    float v[HB][kFusedMergeMax][DPL];
+    float v[HB][kMergeFanIn<D>][DPL];
 #pragma unroll
     for (int hb = 0; hb < HB; ++hb) {
       const float* po = p.part_o + (row0 + h0 + hb) * p.S_max * D + lane * DPL;
 #pragma unroll
-      for (int s = 0; s < kFusedMergeMax; ++s) {
+      for (int s = 0; s < kMergeFanIn<D>; ++s) {
         if (s < nsplit) {
           if constexpr (DPL == 4) {
             const float4 x = __ldcg(reinterpret_cast<const float4*>(po + static_cast<size_t>(s) * D));
@@ -250,7 +360,7 @@ __device__ __forceinline__ void merge_group(const Params& p, int r, int g, int n
 #pragma unroll
       for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
 #pragma unroll
-      for (int s = 0; s < kFusedMergeMax; ++s) {
+      for (int s = 0; s < kMergeFanIn<D>; ++s) {
         const float ws = __shfl_sync(0xffffffffu, w, s);
         if (s < nsplit) {
 #pragma unroll
@@ -273,6 +383,7 @@ __device__ __forceinline__ void merge_group(const Params& p, int r, int g, int n
 template <int D, int G, int NS, int MAXW>
 __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p) {
   using LY = Layout<D, G, NS>;
+  constexpr int kFI = kMergeFanIn<D>;  // merge-tree fan-in
   using CK = Chunk<D>;
   constexpr int kTok = CK::kTokens;
   // score phase: E elements of d per lane (16 at d=128 unless G=8, whose
@@ -301,6 +412,8 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   auto full_bar = [&](int i) { return wbase + LY::kBarOff + 8u * i; };
   ChunkInfo* fifo = reinterpret_cast<ChunkInfo*>(wb + LY::kFifoOff);
   ItemInfo* items = reinterpret_cast<ItemInfo*>(wb + LY::kItemOff);
+  ItemInfo* climb = reinterpret_cast<ItemInfo*>(wb + LY::kClimbOff);
+  if (lane < kClimbSlots) climb[lane].r = -1;
   float* pb = reinterpret_cast<float*>(wb + LY::kPbOff);
 
   if constexpr (!kCpAsync) {
@@ -785,24 +898,25 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
         }
       }
       if (balanced && it.nsplit > 1) {
-        const size_t gi = static_cast<size_t>(it.r) * p.Hkv + it.g;
-        if (it.s == 0 && lane == 0) p.group_splits[gi] = it.nsplit;
-        if (it.nsplit <= kFusedMergeMax) {
-          // the warp that finishes the group's last split merges the partials;
-          // lane 0's release add publishes every lane's partial stores (they
-          // precede it through the warp barrier)
-          __syncwarp();
-          uint32_t done = 0;
-          if (lane == 0) done = atomic_add_release_gpu(p.group_done + gi, 1u);
-          done = __shfl_sync(0xffffffffu, done, 0);
-          if (done == static_cast<uint32_t>(it.nsplit - 1)) {
-            __threadfence();
-            merge_group<D, G>(p, it.r, it.g, it.nsplit, lane);
-            if (lane == 0) p.group_done[gi] = 0;  // ready for the next launch
+        // count this piece in its first-level merge node; the warp that
+        // completes the node merges it: now when it is the tree's top, else
+        // after its slice.  Lane 0's release add publishes every lane's
+        // partial stores (they precede it through the warp barrier).
+        __syncwarp();
+        const int jp = it.s / kFI;
+        uint32_t* c = p.group_done + (static_cast<size_t>(it.r) * p.Hkv + it.g) * p.merge_nodes + jp;
+        uint32_t done = 0;
+        if (lane == 0) done = atomic_add_release_gpu(c, 1u);
+        done = __shfl_sync(0xffffffffu, done, 0);
+        if (done == static_cast<uint32_t>(min(kFI, it.nsplit - jp * kFI) - 1)) {
+          __threadfence();
+          if (lane == 0) *c = 0;  // ready for the next launch
+          if (it.nsplit <= kFI) {
+            merge_regs<D, G>(p, it.r, it.g, it.nsplit, lane);  // a one-level tree: done now
+          } else if (lane == 0) {
+            climb[climb[0].r < 0 ? 0 : 1] = ItemInfo{it.r, it.g, jp, it.nsplit};
           }
         }
-      } else if (balanced && it.s == 0 && lane == 0) {
-        p.group_splits[static_cast<size_t>(it.r) * p.Hkv + it.g] = 1;
       }
     }
   }
@@ -813,6 +927,44 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     }
   } else {
     cp_async_wait<0>();
+  }
+  // merge the first-level tree nodes this warp completed, then climb: node
+  // (level k, index j) of a group cut into n pieces merges children slots
+  // off_{k-1} + [j*fan-in, (j+1)*fan-in) into slot off_k + j (off_0 = 0,
+  // off_{k+1} = off_k + n_k) or, at the top, into the output, and counts its
+  // finished children in counter off_k - n + j
+  __syncwarp();
+#pragma unroll 1
+  for (int e = 0; e < kClimbSlots; ++e) {
+    const ItemInfo cl = climb[e];
+    if (cl.r < 0) continue;
+    __threadfence();  // acquire: lane 0 saw the node's last child arrive
+    const int n = cl.nsplit;
+    uint32_t* ctr = p.group_done + (static_cast<size_t>(cl.r) * p.Hkv + cl.g) * p.merge_nodes;
+    int j = cl.s, nprev = n, offprev = 0, nk = (n + kFI - 1) / kFI, offk = n;
+    for (;;) {
+      const int c0 = j * kFI, cnt = min(kFI, nprev - c0);
+      if (nk == 1) {
+        merge_staged<D, G, NS, true>(p, cl.r, cl.g, offprev + c0, cnt, 0, lane, wbase, reinterpret_cast<const float*>(wb));
+        break;
+      }
+      merge_staged<D, G, NS, false>(p, cl.r, cl.g, offprev + c0, cnt, offk + j, lane, wbase,
+                                   reinterpret_cast<const float*>(wb));
+      const int jp = j / kFI;
+      uint32_t* c = ctr + (offk + nk - n + jp);
+      __syncwarp();
+      uint32_t done = 0;
+      if (lane == 0) done = atomic_add_release_gpu(c, 1u);
+      done = __shfl_sync(0xffffffffu, done, 0);
+      if (done != static_cast<uint32_t>(min(kFI, nk - jp * kFI) - 1)) break;
+      __threadfence();
+      if (lane == 0) *c = 0;  // ready for the next launch
+      nprev = nk;
+      offprev = offk;
+      offk += nk;
+      nk = (nk + kFI - 1) / kFI;
+      j = jp;
+    }
   }
   if (lane == 0) {
     __threadfence();
@@ -827,16 +979,15 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
 // Merge split partials.  One CTA per (request, query head) row; its warps
 // stride over the splits (four splits' loads in flight per warp), each lane
 // owning D/32 columns, and the per-warp sums meet in shared memory.
-// num_splits[row / rows_per_entry] is the row's split count (per request in
-// the standalone combine, per (request, KV head) group after an automatic
-// split); rows with at most skip_below splits are left alone (written by the
-// partition kernel).
+// num_splits[row / Hq] is the row's split count; rows with at most
+// skip_below splits are left alone (a fixed-partition decode writes the
+// unsplit rows itself).
 constexpr int kCombineMaxWarps = 8;
 
 template <int D>
 __global__ void __launch_bounds__(32 * kCombineMaxWarps) combine_kernel(
     const float* __restrict__ part_o, const float* __restrict__ part_lse,
-    const int32_t* __restrict__ num_splits, int32_t rows_per_entry, int32_t S_max,
+    const int32_t* __restrict__ num_splits, int32_t Hq, int32_t S_max,
     uint16_t* __restrict__ out, float* __restrict__ out_lse, int skip_below) {
   constexpr int DPL = D / 32;
   constexpr float kLog2e = 1.4426950408889634f;
@@ -847,7 +998,7 @@ __global__ void __launch_bounds__(32 * kCombineMaxWarps) combine_kernel(
   // launched as a programmatic dependent of the partition kernel: wait for
   // that grid to complete (a no-op when launched normally)
   pdl_wait();
-  int n = num_splits[row / rows_per_entry];
+  int n = num_splits[row / Hq];
   if (n <= skip_below) return;
   n = max(0, min(n, S_max));
   const float* ls = part_lse + row * S_max;

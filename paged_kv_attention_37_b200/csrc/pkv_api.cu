@@ -129,7 +129,7 @@ int combine_warps(int32_t max_splits) {
 // of following its last CTA.
 template <int D>
 int launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits, int32_t B,
-                   int32_t Hq, int32_t rows_per_entry, int32_t S, uint16_t* out, float* out_lse,
+                   int32_t Hq, int32_t S, uint16_t* out, float* out_lse,
                    int skip_below, bool after_decode, cudaStream_t stream) {
   const long long rows = static_cast<long long>(B) * Hq;
   if (rows > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
@@ -143,7 +143,7 @@ int launch_combine(const float* part_o, const float* part_lse, const int32_t* nu
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = after_decode ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, pkv::decode::combine_kernel<D>, part_o, part_lse, num_splits, rows_per_entry, S,
+  if (cudaLaunchKernelEx(&cfg, pkv::decode::combine_kernel<D>, part_o, part_lse, num_splits, Hq, S,
                          out, out_lse, skip_below) != cudaSuccess)
     return PKV_ERR_CUDA;
   return launch_status();
@@ -162,23 +162,38 @@ int32_t max_splits_for(int32_t max_kv_len, int32_t partition_tokens) {
   return (len + partition_tokens - 1) / partition_tokens;
 }
 
-// Workspace: [counters | group_done | num_splits | group_splits | part_lse |
-// part_o].  The first two regions must be zero before the first call; every
-// call that completes leaves them zero (zero_bytes covers them).
-struct WorkspaceLayout {
-  size_t counters = 0, group_done = 0, num_splits = 0, group_splits = 0, part_lse = 0, part_o = 0,
-         total = 0, zero_bytes = 0;
+// Partial slots per (request, query head) row and merge-tree counters per
+// (request, KV head): the automatic split keeps its pieces and the inner
+// levels of the merge tree in the row; a fixed partition keeps its splits.
+struct SplitSlots {
+  int32_t slots = 1, nodes = 0;
 };
 
-WorkspaceLayout workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t S) {
+SplitSlots split_slots(int32_t max_kv_len, int32_t partition_tokens, int32_t head_dim) {
+  SplitSlots ss;
+  const int32_t pieces = max_splits_for(max_kv_len, partition_tokens);
+  const int fan_in = head_dim == 64 ? pkv::decode::kMergeFanIn<64> : pkv::decode::kMergeFanIn<128>;
+  ss.slots = partition_tokens == 0 ? pkv::decode::merge_tree_slots(pieces, fan_in) : pieces;
+  ss.nodes = partition_tokens == 0 ? pkv::decode::merge_tree_nodes(pieces, fan_in) : 0;
+  return ss;
+}
+
+// Workspace: [counters | group_done | num_splits | part_lse | part_o].  The
+// first two regions must be zero before the first call; every call that
+// completes leaves them zero (zero_bytes covers them).
+struct WorkspaceLayout {
+  size_t counters = 0, group_done = 0, num_splits = 0, part_lse = 0, part_o = 0, total = 0, zero_bytes = 0;
+};
+
+WorkspaceLayout workspace_layout(int32_t B, int32_t Hq, int32_t D, SplitSlots ss) {
   WorkspaceLayout w;
   const size_t groups = static_cast<size_t>(B) * Hq;  // Hq bounds the KV heads
+  const int32_t S = ss.slots;
   w.counters = 0;
   w.group_done = 256;
-  w.num_splits = w.group_done + align256(groups * 4);
+  w.num_splits = w.group_done + align256(groups * std::max<int32_t>(ss.nodes, 1) * 4);
   w.zero_bytes = w.num_splits;
-  w.group_splits = w.num_splits + align256(static_cast<size_t>(B) * 4);
-  w.part_lse = w.group_splits + align256(groups * 4);
+  w.part_lse = w.num_splits + align256(static_cast<size_t>(B) * 4);
   w.part_o = w.part_lse + align256(static_cast<size_t>(B) * Hq * S * 4);
   w.total = w.part_o + align256(static_cast<size_t>(B) * Hq * S * D * 4);
   return w;
@@ -237,14 +252,8 @@ int launch_decode(const pkv::decode::Params& prm, int sm_count, cudaStream_t str
     return PKV_ERR_CUDA;
   if (launch_pdl(kernel, dim3(sm_count), dim3(W * 32), smem, stream, prm) != PKV_OK) return PKV_ERR_CUDA;
   if (prm.partition < 0) return PKV_OK;  // every request is one split
-  if (prm.partition == 0) {
-    // automatic split: groups of at most kFusedMergeMax splits were merged in
-    // the partition kernel; the combine kernel takes the longer ones
-    if (prm.S_max <= pkv::decode::kFusedMergeMax) return PKV_OK;
-    return launch_combine<D>(prm.part_o, prm.part_lse, prm.group_splits, prm.B, prm.Hq, G, prm.S_max,
-                             prm.out, prm.out_lse, pkv::decode::kFusedMergeMax, true, stream);
-  }
-  return launch_combine<D>(prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.Hq, prm.S_max,
+  if (prm.partition == 0) return PKV_OK;  // automatic split: merged by the partition kernel's tree
+  return launch_combine<D>(prm.part_o, prm.part_lse, prm.num_splits, prm.B, prm.Hq, prm.S_max,
                            prm.out, prm.out_lse, 1, true, stream);
 }
 
@@ -351,8 +360,7 @@ int pkv_kv_append(const void* k_new, const void* v_new, const int32_t* slot_mapp
 size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t head_dim,
                                   int32_t max_kv_len, int32_t partition_tokens) {
   if (batch < 0 || num_q_heads < 0 || head_dim < 0 || max_kv_len < 0) return 0;
-  const int32_t S = max_splits_for(max_kv_len, partition_tokens);
-  return workspace_layout(batch, num_q_heads, head_dim, S).total;
+  return workspace_layout(batch, num_q_heads, head_dim, split_slots(max_kv_len, partition_tokens, head_dim)).total;
 }
 
 int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool,
@@ -380,8 +388,8 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
       static_cast<long long>(batch) * pool.num_kv_heads * (max_kv / pkv::decode::kPartitionQuantum + 1) >=
           (1ll << 31))
     return PKV_ERR_BAD_SHAPE;
-  const int32_t S = max_splits_for(max_kv, partition_tokens);
-  const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, pool.head_dim, S);
+  const SplitSlots ss = split_slots(max_kv, partition_tokens, pool.head_dim);
+  const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, pool.head_dim, ss);
   if (workspace == nullptr || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
   DeviceInfo dev;
@@ -401,15 +409,15 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   prm.num_splits = reinterpret_cast<int32_t*>(ws + wl.num_splits);
   prm.counters = reinterpret_cast<uint32_t*>(ws + wl.counters);
   prm.group_done = reinterpret_cast<uint32_t*>(ws + wl.group_done);
-  prm.group_splits = reinterpret_cast<int32_t*>(ws + wl.group_splits);
   prm.B = batch;
   prm.Hq = num_q_heads;
   prm.Hkv = pool.num_kv_heads;
   prm.P = pool.page_size;
   prm.max_pages = max_pages;
   prm.num_pages = pool.num_pages;
-  prm.S_max = S;
+  prm.S_max = ss.slots;
   prm.partition = partition_tokens;
+  prm.merge_nodes = ss.nodes;
   prm.scale_log2 = scale * 1.4426950408889634f;
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = prepare_workspace(workspace, wl.zero_bytes, s)) != PKV_OK) return st;
@@ -430,9 +438,9 @@ int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_
   if ((st = current_device(&dev)) != PKV_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if (head_dim == 128)
-    return launch_combine<128>(part_o, part_lse, num_splits, batch, num_q_heads, num_q_heads, max_splits,
+    return launch_combine<128>(part_o, part_lse, num_splits, batch, num_q_heads, max_splits,
                                static_cast<uint16_t*>(out), out_lse, -1, false, s);
-  return launch_combine<64>(part_o, part_lse, num_splits, batch, num_q_heads, num_q_heads, max_splits,
+  return launch_combine<64>(part_o, part_lse, num_splits, batch, num_q_heads, max_splits,
                             static_cast<uint16_t*>(out), out_lse, -1, false, s);
 }
 
@@ -571,9 +579,9 @@ extern "C" int pkv_paged_attn_decode_static(const void* q, int32_t batch, int32_
   // The array keeps whatever the previous call left; the scheduling and
   // per-group split counters at its start must be zero when the decode
   // kernel begins.
-  const size_t zero = workspace_layout(batch, num_q_heads, pool.head_dim,
-                                       max_splits_for(static_cast<int32_t>(max_kv), partition_tokens))
-                          .zero_bytes;
+  const size_t zero =
+      workspace_layout(batch, num_q_heads, pool.head_dim, split_slots(static_cast<int32_t>(max_kv), partition_tokens, pool.head_dim))
+          .zero_bytes;
   if (cudaMemsetAsync(scratch, 0, zero, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return PKV_ERR_CUDA;
   return pkv_paged_attn_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages,

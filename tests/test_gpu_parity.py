@@ -152,6 +152,17 @@ def test_decode_splitk_small(pkv):
     run_decode_case(pkv, w, partitions=(0, 512, 1024, 2048, 4096, -1))
 
 
+@pytest.mark.parametrize("d,L", [(128, 900), (128, 1100), (128, 8100), (128, 8400), (128, 66000),
+                                 (64, 1900), (64, 2200), (64, 33000)])
+def test_decode_auto_merge_tree_levels(pkv, d, L):
+    # one request and one KV head: the automatic split cuts it into slices of
+    # about 128 tokens.  With a fan-in of 8 (d = 128) these lengths give about
+    # 7, 9, 63, 66 and 516 pieces, merge trees of one, two, two, three and four
+    # levels; with 16 (d = 64), about 15, 17 and 258 pieces: one, two, three.
+    w = make_workload("qwen3_decode", 31, lens=[L], num_kv_heads=1, num_q_heads=4, head_dim=d)
+    run_decode_case(pkv, w, partitions=(0,))
+
+
 def test_decode_reuses_workspace(pkv):
     # the scheduling counters in the workspace must return to zero each call
     w = make_workload("qwen3_decode", 8, B=6, len_lo=300, len_hi=3000)
