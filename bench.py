@@ -8,7 +8,7 @@ fragmented large batch, tiny decode).
 
 A step is one pass of the hot path over one batch: kv_append of the step's new
 K/V rows, then attention (chunked prefill for prompt chunks, decode with its
-split-K partition + combine for decode rows).  Inputs are resident in HBM
+split-K partition and in-kernel merge for decode rows).  Inputs are resident in HBM
 when the timed region starts; the KV a step reads is larger than the 126 MB
 L2, so no flush is needed between steps.  Under torchrun each rank runs its
 own batch (requests shard across GPUs with no data-path collective: weak
@@ -219,7 +219,9 @@ class GpuWorkload:
         return self.torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
     def launches_per_step(self):
-        return 1 + (2 if self.dec else 0) + (1 if self.pre else 0)
+        # kv_append, the decode partition kernel (the automatic split merges
+        # in-kernel, no combine launch), the prefill kernel
+        return 1 + (1 if self.dec else 0) + (1 if self.pre else 0)
 
     def step(self, d, ev=None, outs=None):
         """One pass of the hot path on device buffers d; ev optionally brackets
@@ -528,7 +530,7 @@ def main():
         "pct_of_8TBs": 100 * value / HBM_NOMINAL_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": profiled_traffic("decode_partition_qwen3_decode"),
-                     "kernel": "decode split-K partition + combine (one pkv_paged_attn_decode call)",
+                     "kernel": "decode split-K partition with in-kernel merge (one pkv_paged_attn_decode call)",
                      "timing": "CUDA events around each decode call over a second pass of the K timed steps",
                      "peak_source": f"{peak_src} hbm_gbs", "pct_of_8TBs": 100 * achieved / HBM_NOMINAL_GBS},
         "cpu_baseline": ({"value": cpu_rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
