@@ -251,8 +251,11 @@ class GpuWorkload:
         """`steps` steps through the public API from pinned host buffers: every
         step copies its inputs host-to-device, runs the kernels and reads its
         outputs back.  Two buffer sets and a copy stream let the copies of one
-        step overlap the kernels of its neighbours; the caller times the whole
-        run on the current stream (it waits for the copy stream at the end)."""
+        step overlap the kernels of its neighbours: step i+1's inputs are
+        queued on the copy stream before step i's read-back (which waits for
+        step i's kernels), so they land while step i computes.  The caller
+        times the whole run on the current stream (it waits for the copy
+        stream at the end)."""
         torch = self.torch
         main = torch.cuda.current_stream()
         cs = self._copy_stream = getattr(self, "_copy_stream", None) or torch.cuda.Stream()
@@ -260,19 +263,27 @@ class GpuWorkload:
         ev_done = [torch.cuda.Event() for _ in range(2)]
         ev_out = [torch.cuda.Event() for _ in range(2)]
         cs.wait_stream(main)
+
+        def load(i):  # on the copy stream
+            b = i & 1
+            if i >= 2:
+                cs.wait_event(ev_done[b])  # the kernels of step i-2 no longer read set b
+            self.in_dev[b].buf.copy_(self.in_host.buf, non_blocking=True)
+            ev_in[b].record(cs)
+
+        with torch.cuda.stream(cs):
+            if steps > 0:
+                load(0)
         for i in range(steps):
             b = i & 1
-            with torch.cuda.stream(cs):
-                if i >= 2:
-                    cs.wait_event(ev_done[b])  # the kernels of step i-2 no longer read set b
-                self.in_dev[b].buf.copy_(self.in_host.buf, non_blocking=True)
-                ev_in[b].record(cs)
             main.wait_event(ev_in[b])
             if i >= 2:
                 main.wait_event(ev_out[b])  # step i-2's outputs have left set b
             self.step(self.dev_sets[b], outs=self.out_sets[b])
             ev_done[b].record(main)
             with torch.cuda.stream(cs):
+                if i + 1 < steps:
+                    load(i + 1)
                 cs.wait_event(ev_done[b])
                 self.out_host[b].buf.copy_(self.out_dev[b].buf, non_blocking=True)
                 ev_out[b].record(cs)
