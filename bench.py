@@ -339,17 +339,37 @@ def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    # timed region: K whole steps, nothing recorded between the kernels (an
-    # event between two launches would serialise them and cost the
-    # programmatic-dependent-launch overlap)
+    # timed region: K whole steps captured once as one CUDA graph, as a
+    # serving loop replays its decode step, with nothing recorded between the
+    # kernels (an event between two launches would serialise them and cost
+    # the programmatic-dependent-launch overlap); one untimed replay uploads
+    # the graph.  Where capture is refused, the K steps run eagerly.
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(steps):
+                g.step(g.dev)
+        graph.replay()
+        torch.cuda.synchronize()
+    except Exception as e:  # noqa: BLE001
+        graph, graph_err = None, repr(e)[:200]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
     t0, t1 = mk(), mk()
     with ClockSampler(clocks_index) as clk:
         t0.record()
-        for i in range(steps):
-            g.step(g.dev)
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(steps):
+                g.step(g.dev)
         t1.record()
         torch.cuda.synchronize()
     total_ms = max_over_ranks(dist, t0.elapsed_time(t1))
+    timing = "one CUDA graph of the K steps" if graph is not None else f"eager launches ({graph_err})"
+    del graph
     # second timed pass of K steps with CUDA events around each attention call
     # on its stream: the per-call kernel durations of the roofline
     torch.cuda.synchronize()
@@ -382,6 +402,7 @@ def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
         "kv_bytes_dec": w.kv_bytes_read(w.decode_ids), "kv_bytes_pre": w.kv_bytes_read(w.prefill_ids),
         "tokens": int(w.new_lens.sum()), "flops_pre": prefill_flops(w),
         "launches": g.launches_per_step(), "clocks": clk.summary(), "h2d": h2d, "d2h": d2h,
+        "timing": timing,
     }
     del g
     torch.cuda.empty_cache()
@@ -502,7 +523,7 @@ def main():
         if args.workloads == "all" else [n for n in args.workloads.split(",") if n])
     for n in names:
         r = measure(pkv, torch, n, args.steps, args.warmup, dist, local)
-        e = {"ms_per_step": r["ms_per_step"], "tokens_per_step": r["tokens"],
+        e = {"ms_per_step": r["ms_per_step"], "timed_region": r["timing"], "tokens_per_step": r["tokens"],
              "tokens_per_s": world * r["tokens"] / (r["ms_per_step"] / 1e3),
              "e2e_ms_per_step": r["e2e_ms_per_step"]}
         if r["dec_ms"]:
@@ -537,7 +558,8 @@ def main():
         "data": "synthetic",
         "config": {"workload": HEADLINE, **{k: v for k, v in w.describe().items() if k != "workload"},
                    "kv_bytes_per_step": kv_bytes, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (KV read per step > 126 MB), no flush"},
+                   "l2": "inputs larger than L2 (KV read per step > 126 MB), no flush",
+                   "timed_region": head["timing"]},
         "pct_of_8TBs": 100 * value / HBM_NOMINAL_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": profiled_traffic("decode_partition_qwen3_decode"),
