@@ -76,6 +76,34 @@ def test_workspace_size(lib):
     assert f(-1, 32, 64, 10, 0) == 0
 
 
+def test_workspace_holds_the_merge_tree(lib):
+    # Under the automatic split a (request, KV head) group is cut into at most
+    # n = ceil(L / 128) + 1 pieces; the pieces and every inner level of their
+    # merge tree (fan-in 8 at d = 128, 16 at d = 64: each level a ceiling
+    # division of the one below, until one node is left) need partial slots.
+    lib.pkv_decode_workspace_bytes.restype = ctypes.c_size_t
+    f = lib.pkv_decode_workspace_bytes
+
+    def slots(n, fan):
+        levels = [n]
+        while levels[-1] > 1:
+            levels.append(-(-levels[-1] // fan))
+        return sum(levels[:-1]) if len(levels) > 1 else 1
+
+    B, Hq = 3, 32
+    prev = 0
+    for d, fan in ((128, 8), (64, 16)):
+        for L in (1, 100, 1000, 1024, 1025, 8192, 8193, 65536, 131072):
+            n = -(-L // 128) + 1
+            got = f(B, Hq, d, L, 0)
+            assert got >= B * Hq * slots(n, fan) * (d + 1) * 4, (d, L)
+            if d == 128:
+                assert got >= prev  # grows with the longest context
+                prev = got
+    # a tree of more than one level holds more than its pieces alone
+    assert slots(9, 8) == 9 + 2 and slots(65, 8) == 65 + 9 + 2 and slots(8, 8) == 8
+
+
 def test_host_validation_without_gpu(lib):
     good = PoolDesc(64, 16, 8, 128)
     dummy = ctypes.c_void_p(16)
