@@ -160,10 +160,11 @@ PKV_API size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, in
  *
  * Requests that are not split are written by the partition kernel directly.
  * Split ones go through fp32 partials.  With the automatic split, the pieces
- * of a (request, KV head) are merged inside the partition kernel by a tree of
- * merges of at most 8 partials each, every node merged by the warp that
- * finishes its last child, so one kernel does the whole call.  With a fixed
- * partition, a second, combine kernel merges the split requests.
+ * of a (request, KV head) are merged inside the partition kernel by a tree
+ * of merges of at most 8 (d = 128) or 16 (d = 64) partials each, every node
+ * merged by the warp that finishes its last child, so one kernel does the
+ * whole call.  With a fixed partition, a second, combine kernel merges the
+ * split requests.
  */
 PKV_API int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads,
                           const void* k_pool, const void* v_pool, pkv_pool_desc pool,
