@@ -29,7 +29,7 @@ What it computes, and where the pages define it:
   "Flash-Decoding": a long context is cut along the KV length into
   partitions whose partial results are then combined.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   R1  query head h uses KV head h // G (contiguous groups);
   R2  a decode request's kv_len counts the token appended this step, whose
       query sits at position kv_len - 1; a prefill chunk of n rows after c
