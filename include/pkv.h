@@ -95,8 +95,8 @@ enum pkv_status {
 /* Bits of the device-side error word (see pkv_device_error_flags). */
 #define PKV_FLAG_WAIT_TIMEOUT   0x1u  /* a pipeline wait hit its ~2 s limit; the kernel gave up */
 #define PKV_FLAG_BAD_LENGTH     0x2u  /* a kv_len/ctx/chunk length < 0 or beyond max_pages*page_size */
-#define PKV_FLAG_BAD_SLOT       0x4u  /* kv_append slot >= num_pages*page_size (row skipped) */
-#define PKV_FLAG_BAD_QUERY_ROWS 0x8u  /* cu_q_lens not non-decreasing within [0, total_q] */
+#define PKV_FLAG_BAD_SLOT       0x4u  /* kv_append slot < -1 or >= num_pages*page_size (row skipped) */
+#define PKV_FLAG_BAD_QUERY_ROWS 0x8u  /* cu_q_lens not non-decreasing within [0, total_q], or a chunk longer than max_q_len */
 #define PKV_FLAG_BAD_PAGE       0x10u /* a page-table entry outside [0, num_pages) was seen (page 0 or zeros read instead) */
 #define PKV_FLAG_INTERNAL       0x20u /* a kernel found an internal invariant broken and skipped its work */
 
@@ -112,8 +112,9 @@ enum pkv_status {
  *   k_pool, v_pool pools as above, written in place
  *
  * A pure bit copy: each pool row equals its source row bit for bit.  Slots
- * beyond the pool raise PKV_FLAG_BAD_SLOT and are skipped.  Two rows with the
- * same slot race (one of them wins).  num_tokens == 0 launches nothing.
+ * beyond the pool, and negative slots other than -1, raise PKV_FLAG_BAD_SLOT
+ * and are skipped.  Two rows with the same slot race (one of them wins).
+ * num_tokens == 0 launches nothing.
  */
 PKV_API int pkv_kv_append(const void* k_new, const void* v_new, const int32_t* slot_mapping,
                   int32_t num_tokens, void* k_pool, void* v_pool, pkv_pool_desc pool,
@@ -203,7 +204,9 @@ PKV_API int pkv_split_k_combine(const float* part_o, const float* part_lse, cons
  *                cu_q_lens[r] .. cu_q_lens[r+1]-1
  *   cu_q_lens    [batch+1] int32, non-decreasing, cu_q_lens[0] = 0,
  *                cu_q_lens[batch] <= total_q
- *   max_q_len    an upper bound on any chunk length (sizes the grid)
+ *   max_q_len    an upper bound on any chunk length (sizes the grid); a
+ *                chunk longer than it raises PKV_FLAG_BAD_QUERY_ROWS and its
+ *                rows are not written
  *   ctx_offsets  [batch] int32: tokens of request r before its chunk; chunk
  *                row i sits at position ctx_offsets[r] + i and sees keys
  *                0 .. ctx_offsets[r] + i (diagonal included)

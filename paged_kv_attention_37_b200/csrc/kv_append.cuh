@@ -31,8 +31,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict_
     const int h = static_cast<int>(row % num_kv_heads);
     const int64_t t = row / num_kv_heads;
     const int32_t slot = __ldg(slots + t);
-    if (slot < 0) continue;  // padding row
-    if (slot >= num_slots) {
+    if (slot == -1) continue;  // padding row
+    if (slot < 0 || slot >= num_slots) {  // not a slot of this pool: skipped, flagged
       if (c == 0 && h == 0) raise_flag(PKV_FLAG_BAD_SLOT);
       continue;
     }

@@ -105,6 +105,11 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     return;
   }
   const int n_qt = (n_r + QPOS - 1) / QPOS;
+  if (n_qt > p.qtiles) {
+    // a chunk longer than the max_q_len the grid was sized for: refused whole
+    if (g == 0 && qt_rev == 0 && threadIdx.x == 0) raise_flag(PKV_FLAG_BAD_QUERY_ROWS);
+    return;
+  }
   if (qt_rev >= n_qt) return;
   const int qt = n_qt - 1 - qt_rev;
   const int c = p.ctx_offsets[r];
