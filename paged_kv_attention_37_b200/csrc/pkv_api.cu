@@ -220,6 +220,14 @@ int prepare_workspace(void* ws, size_t need, cudaStream_t stream) {
   return PKV_OK;
 }
 
+// Record that the first `bytes` of workspace ws are zero (the caller has
+// just cleared them on the stream the next call uses).
+void mark_workspace_zero(void* ws, size_t bytes) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_ws_zero.find(ws) == g_ws_zero.end() && g_ws_zero.size() >= kMaxTrackedWorkspaces) g_ws_zero.clear();
+  g_ws_zero[ws] = bytes;
+}
+
 // ------------------------------------------------------------ decode launch
 template <int D, int G>
 int launch_decode(const pkv::decode::Params& prm, int sm_count, cudaStream_t stream) {
@@ -309,6 +317,83 @@ int dispatch_prefill_group(int group, const pkv::prefill::Params& prm, const CUt
   return PKV_ERR_UNSUPPORTED;
 }
 
+// Host-side checks shared by both decode entry points, and the split and
+// workspace layout the call implies.  Returns PKV_OK for an empty batch
+// before the pointer checks (nothing will be launched).
+struct DecodePlan {
+  int group = 0;
+  SplitSlots ss;
+  WorkspaceLayout wl;
+};
+
+int check_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool, const void* v_pool,
+                 const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages,
+                 const int32_t* kv_lens, float scale, int32_t partition_tokens, const void* out,
+                 DecodePlan* dp) {
+  if (batch < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
+  int st = check_pool(pool);
+  if (st != PKV_OK) return st;
+  if ((st = check_heads(num_q_heads, pool, &dp->group)) != PKV_OK) return st;
+  if (partition_tokens > 0 &&
+      (partition_tokens % pkv::decode::kPartitionQuantum != 0 || partition_tokens > 65536))
+    return PKV_ERR_BAD_SHAPE;
+  if (partition_tokens < -1) return PKV_ERR_BAD_SHAPE;
+  if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
+  if (!std::isfinite(scale)) return PKV_ERR_BAD_SHAPE;
+  const int32_t max_kv = max_pages * pool.page_size;
+  // the automatic split counts the batch's token-heads in 32-token quanta (int32)
+  if (partition_tokens == 0 &&
+      static_cast<long long>(batch) * pool.num_kv_heads * (max_kv / pkv::decode::kPartitionQuantum + 1) >=
+          (1ll << 31))
+    return PKV_ERR_BAD_SHAPE;
+  dp->ss = split_slots(max_kv, partition_tokens, pool.head_dim);
+  dp->wl = workspace_layout(batch, num_q_heads, pool.head_dim, dp->ss);
+  if (batch == 0) return PKV_OK;
+  if (!q || !k_pool || !v_pool || !page_table || !kv_lens || !out) return PKV_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return PKV_ERR_MISALIGNED;
+  return PKV_OK;
+}
+
+// Launch a checked decode call on workspace ws (at least dp.wl.total bytes,
+// 256-byte aligned).
+int run_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool, const void* v_pool,
+               const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages,
+               const int32_t* kv_lens, float scale, int32_t partition_tokens, const DecodePlan& dp,
+               void* workspace, void* out, float* out_lse, cudaStream_t s) {
+  DeviceInfo dev;
+  int st;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  const WorkspaceLayout& wl = dp.wl;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  pkv::decode::Params prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.k_pool = static_cast<const uint16_t*>(k_pool);
+  prm.v_pool = static_cast<const uint16_t*>(v_pool);
+  prm.page_table = page_table;
+  prm.kv_lens = kv_lens;
+  prm.out = static_cast<uint16_t*>(out);
+  prm.out_lse = out_lse;
+  prm.part_o = reinterpret_cast<float*>(ws + wl.part_o);
+  prm.part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
+  prm.num_splits = reinterpret_cast<int32_t*>(ws + wl.num_splits);
+  prm.counters = reinterpret_cast<uint32_t*>(ws + wl.counters);
+  prm.group_done = reinterpret_cast<uint32_t*>(ws + wl.group_done);
+  prm.B = batch;
+  prm.Hq = num_q_heads;
+  prm.Hkv = pool.num_kv_heads;
+  prm.P = pool.page_size;
+  prm.max_pages = max_pages;
+  prm.num_pages = pool.num_pages;
+  prm.S_max = dp.ss.slots;
+  prm.partition = partition_tokens;
+  prm.merge_nodes = dp.ss.nodes;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  if ((st = prepare_workspace(workspace, wl.zero_bytes, s)) != PKV_OK) return st;
+  if (pool.head_dim == 128) return dispatch_decode_group<128>(dp.group, prm, dev.sm_count, s);
+  return dispatch_decode_group<64>(dp.group, prm, dev.sm_count, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -368,61 +453,14 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
                           int32_t max_pages, const int32_t* kv_lens, float scale,
                           int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                           void* out, float* out_lse, pkv_stream_t stream) {
-  if (batch < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
-  int st = check_pool(pool);
-  if (st != PKV_OK) return st;
-  int group = 0;
-  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
-  if (partition_tokens > 0 &&
-      (partition_tokens % pkv::decode::kPartitionQuantum != 0 || partition_tokens > 65536))
-    return PKV_ERR_BAD_SHAPE;
-  if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
-  if (!std::isfinite(scale)) return PKV_ERR_BAD_SHAPE;
-  if (batch == 0) return PKV_OK;
-  if (!q || !k_pool || !v_pool || !page_table || !kv_lens || !out) return PKV_ERR_NULL_POINTER;
-  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
-    return PKV_ERR_MISALIGNED;
-  const int32_t max_kv = max_pages * pool.page_size;
-  // the automatic split counts the batch's token-heads in 32-token quanta (int32)
-  if (partition_tokens == 0 &&
-      static_cast<long long>(batch) * pool.num_kv_heads * (max_kv / pkv::decode::kPartitionQuantum + 1) >=
-          (1ll << 31))
-    return PKV_ERR_BAD_SHAPE;
-  const SplitSlots ss = split_slots(max_kv, partition_tokens, pool.head_dim);
-  const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, pool.head_dim, ss);
-  if (workspace == nullptr || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
+  DecodePlan dp;
+  const int st = check_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens,
+                              scale, partition_tokens, out, &dp);
+  if (st != PKV_OK || batch == 0) return st;
+  if (workspace == nullptr || workspace_bytes < dp.wl.total) return PKV_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != PKV_OK) return st;
-  const int D = pool.head_dim;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  pkv::decode::Params prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.k_pool = static_cast<const uint16_t*>(k_pool);
-  prm.v_pool = static_cast<const uint16_t*>(v_pool);
-  prm.page_table = page_table;
-  prm.kv_lens = kv_lens;
-  prm.out = static_cast<uint16_t*>(out);
-  prm.out_lse = out_lse;
-  prm.part_o = reinterpret_cast<float*>(ws + wl.part_o);
-  prm.part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
-  prm.num_splits = reinterpret_cast<int32_t*>(ws + wl.num_splits);
-  prm.counters = reinterpret_cast<uint32_t*>(ws + wl.counters);
-  prm.group_done = reinterpret_cast<uint32_t*>(ws + wl.group_done);
-  prm.B = batch;
-  prm.Hq = num_q_heads;
-  prm.Hkv = pool.num_kv_heads;
-  prm.P = pool.page_size;
-  prm.max_pages = max_pages;
-  prm.num_pages = pool.num_pages;
-  prm.S_max = ss.slots;
-  prm.partition = partition_tokens;
-  prm.merge_nodes = ss.nodes;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  auto s = reinterpret_cast<cudaStream_t>(stream);
-  if ((st = prepare_workspace(workspace, wl.zero_bytes, s)) != PKV_OK) return st;
-  if (D == 128) return dispatch_decode_group<128>(group, prm, dev.sm_count, s);
-  return dispatch_decode_group<64>(group, prm, dev.sm_count, s);
+  return run_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens, scale,
+                    partition_tokens, dp, workspace, out, out_lse, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
@@ -557,34 +595,23 @@ extern "C" int pkv_paged_attn_decode_static(const void* q, int32_t batch, int32_
                                             int32_t max_pages, const int32_t* kv_lens, float scale,
                                             int32_t partition_tokens, void* out, float* out_lse,
                                             pkv_stream_t stream) {
-  // the argument checks of pkv_paged_attn_decode, so that a bad call leaves
-  // the scratch untouched
-  if (batch < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
-  int st = check_pool(pool);
+  // every argument check of pkv_paged_attn_decode comes first, so that a
+  // refused call leaves the scratch untouched
+  DecodePlan dp;
+  int st = check_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens, scale,
+                        partition_tokens, out, &dp);
   if (st != PKV_OK) return st;
-  int group = 0;
-  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
-  const long long max_kv = static_cast<long long>(max_pages) * pool.page_size;
-  if (max_kv > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
-  if (batch > 0 && (!q || !k_pool || !v_pool || !page_table || !kv_lens || !out))
-    return PKV_ERR_NULL_POINTER;
-  if (batch > 0 && (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out)))
-    return PKV_ERR_MISALIGNED;
-  const size_t need = pkv_decode_workspace_bytes(batch, num_q_heads, pool.head_dim,
-                                                 static_cast<int32_t>(max_kv), partition_tokens);
-  if (need > kStaticScratchBytes) return PKV_ERR_WORKSPACE;  // beyond the built-in 32 MiB
+  if (dp.wl.total > kStaticScratchBytes) return PKV_ERR_WORKSPACE;  // beyond the built-in 32 MiB
   if (batch == 0) return PKV_OK;
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != PKV_OK) return st;
   // The array keeps whatever the previous call left; the scheduling and
   // per-group split counters at its start must be zero when the decode
-  // kernel begins.
-  const size_t zero =
-      workspace_layout(batch, num_q_heads, pool.head_dim, split_slots(static_cast<int32_t>(max_kv), partition_tokens, pool.head_dim))
-          .zero_bytes;
-  if (cudaMemsetAsync(scratch, 0, zero, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return PKV_ERR_CUDA;
-  return pkv_paged_attn_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages,
-                               kv_lens, scale, partition_tokens, scratch, kStaticScratchBytes, out,
-                               out_lse, stream);
+  // kernel begins.  Having cleared them here, record them as clear so the
+  // shared launch path does not clear them a second time.
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, dp.wl.zero_bytes, s) != cudaSuccess) return PKV_ERR_CUDA;
+  mark_workspace_zero(scratch, dp.wl.zero_bytes);
+  return run_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens, scale,
+                    partition_tokens, dp, scratch, out, out_lse, s);
 }

@@ -134,6 +134,18 @@ def test_host_validation_without_gpu(lib):
     # non-finite scale
     assert dec(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, float("nan"), 0, ws, 1 << 20, dummy, None, None) == -2
 
+    # the scratch-free entry point runs the same checks before touching its scratch
+    lib.pkv_paged_attn_decode_static.argtypes = [P, I32, I32, P, P, PoolDesc, P, I32, P, ctypes.c_float,
+                                                 I32, P, P, P]
+    sdec = lib.pkv_paged_attn_decode_static
+    assert sdec(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 33, dummy, None, None) == -2
+    assert sdec(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 65536 + 32, dummy, None, None) == -2
+    assert sdec(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, float("inf"), 0, dummy, None, None) == -2
+    assert sdec(dummy, 4, 12, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, dummy, None, None) == -2
+    assert sdec(None, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, dummy, None, None) == -1
+    # a partition below -1 is not one of the documented values
+    assert dec(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, -5, ws, 1 << 20, dummy, None, None) == -2
+
     lib.pkv_paged_attn_chunked_prefill.argtypes = [P, P, I32, I32, I32, I32, P, P, P, PoolDesc, P,
                                                    I32, ctypes.c_float, P, P]
     pre = lib.pkv_paged_attn_chunked_prefill

@@ -6,8 +6,8 @@ are handed only their input and output buffers, servers that must not grow
 their device footprint after start-up.  It keeps the split-K scratch in a
 fixed 32 MiB array inside the library instead of a caller workspace.  These
 tests call it through the C ABI and check that two calls in a row give the
-same results as the regular entry point, within the parity tolerance, and
-that sizes beyond the array are refused.  The file is named to be collected
+same results as the regular entry point, within the parity tolerance and bit
+for bit, and that sizes beyond the array and bad partitions are refused.  The file is named to be collected
 last, and it builds all of its own inputs, so it passes alone in a fresh
 process as well as after the other tests.
 """
@@ -49,7 +49,26 @@ def test_static_scratch_decode_matches_workspace_decode(partition):
         torch.cuda.synchronize()
         _close(out, ref, f"output, call {call}")
         _close(lse, ref_lse, f"lse, call {call}")
+        # the same kernels on the same inputs: the split plan and every merge
+        # order are fixed by the shapes, so the results agree bit for bit
+        assert torch.equal(out, ref), f"output bits, call {call}"
+        assert torch.equal(lse, ref_lse), f"lse bits, call {call}"
     assert pkv.pkv_device_error_flags(clear=True) == 0
+
+
+def test_static_scratch_refuses_bad_partition():
+    import paged_kv_attention_37_b200 as pkv
+
+    # a partition that is not a multiple of 32 is refused before the scratch
+    # is touched, like the workspace entry point refuses it
+    B, hq, hkv, d, P = 2, 8, 2, 128, 16
+    q = torch.zeros((B, hq, d), dtype=torch.bfloat16, device="cuda")
+    pool = torch.zeros((4, hkv, P, d), dtype=torch.bfloat16, device="cuda")
+    table = torch.zeros((B, 4), dtype=torch.int32, device="cuda")
+    lens = torch.ones((B,), dtype=torch.int32, device="cuda")
+    with pytest.raises(pkv.PkvError) as e:
+        pkv.pkv_paged_attn_decode_static(q, pool, pool, table, lens, 0.1, 33)
+    assert e.value.status == -2  # PKV_ERR_BAD_SHAPE
 
 
 def test_static_scratch_refuses_oversized_requests():
