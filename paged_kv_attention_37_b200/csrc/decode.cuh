@@ -512,15 +512,18 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   // let a dependent launch (the combine kernel) be scheduled now; it waits
   // for this whole grid to finish before reading anything
   pdl_launch_dependents();
-  const int part = misc[0], nF = misc[1], total = misc[1] + misc[2];
-  // automatic split: warp w < Weff (= misc[0]) takes quanta
-  // [floor(w*Q/Weff), floor((w+1)*Q/Weff)); the slice holding quantum x is
-  // floor(((x+1)*Weff - 1) / Q)
+  // misc[0] is the partition length of a fixed partition, or under the
+  // automatic split the number of warps that get a slice (Weff)
+  const int part = balanced ? 0 : misc[0], weff = balanced ? misc[0] : 0;
+  const int nF = misc[1], total = misc[1] + misc[2];
+  // automatic split: warp w < Weff takes quanta [floor(w*Q/Weff),
+  // floor((w+1)*Q/Weff)) of the Q = nF quanta; the slice holding quantum x
+  // is floor(((x+1)*Weff - 1) / Q)
   const int wid = blockIdx.x * W + warp;
-  auto slice_start = [&](int w) { return static_cast<int>(static_cast<long long>(w) * nF / part); };
-  auto slice_of = [&](int x) { return static_cast<int>((static_cast<long long>(x + 1) * part - 1) / nF); };
-  int bq = balanced && wid < part ? slice_start(wid) : 0;
-  const int bq_end = balanced && wid < part ? slice_start(wid + 1) : 0;
+  auto slice_start = [&](int w) { return static_cast<int>(static_cast<long long>(w) * nF / weff); };
+  auto slice_of = [&](int x) { return static_cast<int>((static_cast<long long>(x + 1) * weff - 1) / nF); };
+  int bq = balanced && wid < weff ? slice_start(wid) : 0;
+  const int bq_end = balanced && wid < weff ? slice_start(wid + 1) : 0;
 
   // ================= issue side: item cursor, lane 0 issues TMA =================
   bool more = true, active = false;

@@ -101,6 +101,21 @@ def test_kv_append_out_of_range_slot_flags(pkv):
     assert (got[0, 0, 3] == 0x3F80).all() and (got.reshape(-1) != 0).sum() == 64
 
 
+def test_kv_append_negative_slots(pkv):
+    # -1 is padding (skipped, no flag); any other negative slot is not a slot
+    # of the pool: the row is skipped and PKV_FLAG_BAD_SLOT raised
+    kp = torch.zeros((2, 1, 16, 64), dtype=torch.bfloat16, device="cuda")
+    vp = torch.zeros_like(kp)
+    k = torch.ones((3, 1, 64), dtype=torch.bfloat16, device="cuda")
+    pkv.pkv_kv_append(k, k, dev_i32([-1, 5, -1]), kp, vp)
+    assert pkv.pkv_device_error_flags(clear=True) == 0
+    pkv.pkv_kv_append(k, k, dev_i32([-7, 6, -2]), kp, vp)
+    assert pkv.pkv_device_error_flags(clear=True) & pkv.FLAG_BAD_SLOT
+    got = host_bits(kp).reshape(2 * 16, 64)
+    assert (got[5] == 0x3F80).all() and (got[6] == 0x3F80).all()
+    assert (np.delete(got, [5, 6], axis=0) == 0).all()
+
+
 # ------------------------------------------------------------------ decode
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_decode_tiny(pkv, seed):
@@ -141,14 +156,16 @@ def test_decode_group_and_head_dim(pkv, group, d):
     run_decode_case(pkv, w, partitions=(0, -1, 64))
 
 
-def test_decode_page32_fragmented_small(pkv):
-    w = make_workload("frag_large", 3, B=24, median=300.0, max_len=2000)
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_decode_page32_fragmented_small(pkv, seed):
+    w = make_workload("frag_large", seed, B=24, median=300.0, max_len=2000)
     assert w.page_size == 32
     run_decode_case(pkv, w, partitions=(0, -1, 128))
 
 
-def test_decode_splitk_small(pkv):
-    w = make_workload("splitk_long", 2, lens=[4000, 8192 + 13, 20000, 33])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_decode_splitk_small(pkv, seed):
+    w = make_workload("splitk_long", seed, lens=[4000, 8192 + 13, 20000, 33])
     run_decode_case(pkv, w, partitions=(0, 512, 1024, 2048, 4096, -1))
 
 
@@ -255,6 +272,30 @@ def test_prefill_group_and_head_dim(pkv, group, d):
     run_prefill_case(pkv, w)
 
 
+def test_prefill_chunk_longer_than_max_q_len(pkv):
+    # the grid is sized from max_q_len: a longer chunk is refused whole (its
+    # rows keep their contents) and PKV_FLAG_BAD_QUERY_ROWS is raised; the
+    # other request is computed as usual
+    w = make_workload("mixed_prefill_decode", 12, n_prefill=2, chunks=[300, 20], ctx_hi=200,
+                      n_decode=1)
+    ds = DeviceStep(pkv, w)
+    os_ = OracleStep(w)
+    ds.append()
+    os_.append()
+    ref, _, rows = os_.prefill()
+    pre = list(w.prefill_ids)
+    cu = w.cu_q_lens(pre)
+    out = torch.full_like(ds.q_pre, 7.0)
+    pkv.pkv_paged_attn_chunked_prefill(ds.q_pre, ds.cu_q, ds.ctx_pre, ds.k_pool, ds.v_pool, ds.pt_pre,
+                                       w.scale, 64, out=out)
+    assert pkv.pkv_device_error_flags(clear=True) & pkv.FLAG_BAD_QUERY_ROWS
+    got = bf16_to_f64(out)
+    long_r = int(np.argmax(np.diff(cu)))
+    short_rows = np.arange(cu[1 - long_r], cu[2 - long_r])
+    assert (got[cu[long_r]:cu[long_r + 1]] == 7.0).all()
+    assert_close(got[short_rows], ref[short_rows], "prefill, the chunk within max_q_len")
+
+
 def test_prefill_page32(pkv):
     w = make_workload("mixed_prefill_decode", 10, n_prefill=2, chunks=[256, 90], ctx_hi=700,
                       n_decode=1, page_size=32)
@@ -273,29 +314,34 @@ def sample_ids(w, k, rng_seed=0):
 
 
 @pytest.mark.slow
-def test_full_qwen3_decode_sampled(pkv):
-    w = make_workload("qwen3_decode", 0)
-    run_decode_case(pkv, w, ids=sample_ids(w, 6), partitions=(0,))
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_full_qwen3_decode_sampled(pkv, seed):
+    w = make_workload("qwen3_decode", seed)
+    run_decode_case(pkv, w, ids=sample_ids(w, 6, seed), partitions=(0,))
 
 
 @pytest.mark.slow
-def test_full_splitk_long_sampled(pkv):
-    w = make_workload("splitk_long", 0)
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_full_splitk_long_sampled(pkv, seed):
+    w = make_workload("splitk_long", seed)
+    # the shortest and the longest request (32 768 and 131 072 tokens)
     run_decode_case(pkv, w, ids=[0, 3], partitions=(0, 512, 4096))
 
 
 @pytest.mark.slow
-def test_full_frag_large_sampled(pkv):
-    w = make_workload("frag_large", 0)
-    run_decode_case(pkv, w, ids=sample_ids(w, 6), partitions=(0,))
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_full_frag_large_sampled(pkv, seed):
+    w = make_workload("frag_large", seed)
+    run_decode_case(pkv, w, ids=sample_ids(w, 6, seed), partitions=(0,))
 
 
 @pytest.mark.slow
-def test_full_mixed_sampled(pkv):
-    w = make_workload("mixed_prefill_decode", 0)
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_full_mixed_sampled(pkv, seed):
+    w = make_workload("mixed_prefill_decode", seed)
     pre = list(w.prefill_ids)
     by_ctx = sorted(pre, key=lambda r: w.ctx_lens[r])
-    ids = [by_ctx[0], by_ctx[-1]] + sample_ids(w, 3)
+    ids = [by_ctx[0], by_ctx[-1]] + sample_ids(w, 3, seed)
     ds, os_ = run_prefill_case(pkv, w, ids=ids)
     ref, _, sel = os_.decode()
     assert_close(bf16_to_f64(ds.decode())[sel], ref[sel], "mixed decode part")
