@@ -512,9 +512,10 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   // let a dependent launch (the combine kernel) be scheduled now; it waits
   // for this whole grid to finish before reading anything
   pdl_launch_dependents();
-  // misc[0] is the partition length of a fixed partition, or under the
-  // automatic split the number of warps that get a slice (Weff)
-  const int part = balanced ? 0 : misc[0], weff = balanced ? misc[0] : 0;
+  // misc[0] holds one value with two readings: under a fixed partition its
+  // length in tokens (part), under the automatic split the number of warps
+  // that get a slice (weff)
+  const int part = misc[0], weff = part;
   const int nF = misc[1], total = misc[1] + misc[2];
   // automatic split: warp w < Weff takes quanta [floor(w*Q/Weff),
   // floor((w+1)*Q/Weff)) of the Q = nF quanta; the slice holding quantum x
