@@ -99,6 +99,7 @@ enum pkv_status {
 #define PKV_FLAG_BAD_QUERY_ROWS 0x8u  /* cu_q_lens not non-decreasing within [0, total_q], or a chunk longer than max_q_len */
 #define PKV_FLAG_BAD_PAGE       0x10u /* a page-table entry outside [0, num_pages) was seen (page 0 or zeros read instead) */
 #define PKV_FLAG_INTERNAL       0x20u /* a kernel found an internal invariant broken and skipped its work */
+#define PKV_FLAG_NO_FREE_PAGE   0x40u /* copy-on-write append found the free page list exhausted */
 
 /*
  * pkv_kv_append -- write the K/V rows of this step's new tokens into pool
@@ -255,6 +256,77 @@ PKV_API int pkv_paged_attn_decode_static(const void* q, int32_t batch, int32_t n
                                          int32_t max_pages, const int32_t* kv_lens, float scale,
                                          int32_t partition_tokens, void* out, float* out_lse,
                                          pkv_stream_t stream);
+
+/*
+ * pkv_qk_norm_rope_append -- the step before attention in one kernel: the
+ * separate RMSNorm of each projected query and key head row, rotary position
+ * encoding of both, and the write of the new K row (and the V row, as it is)
+ * into the pool (tiny-llm source reading, week 1: Qwen3's "independent
+ * RMSNorm of Q and K after projection" and RoPE; week 2 and the tiny-llm
+ * blog, week 2: RMSNorm and RoPE fused into one kernel to save memory round
+ * trips).
+ *
+ *   q            [num_tokens][Hq][d] bf16, the projected queries
+ *   k, v         [num_tokens][Hkv][d] bf16, the projected keys and values
+ *   q_norm_weight, k_norm_weight  [d] bf16, one weight per element, shared
+ *                by the heads: row x -> x / sqrt(mean(x^2) + eps) * w
+ *   positions    [num_tokens] int32, the position of each token (a decode
+ *                token sits at kv_len - 1, chunk row i at ctx + i)
+ *   slot_mapping [num_tokens] int32, the pool slot of each token's K/V row,
+ *                -1 = skip (as pkv_kv_append)
+ *   rope_theta   RoPE base (> 1): element i pairs with element i + d/2 and
+ *                the pair turns by position * rope_theta^(-2i/d)
+ *   q_out        [num_tokens][Hq][d] bf16, the normalised, rotated queries
+ *                (may be q itself)
+ *
+ * Arithmetic is fp32 from the bf16 inputs, rounded once to bf16; the
+ * rotation angles are formed in fp64.  Bad slots raise PKV_FLAG_BAD_SLOT and
+ * skip the K/V write (the query row is still written).
+ */
+PKV_API int pkv_qk_norm_rope_append(const void* q, const void* k, const void* v, int32_t num_tokens,
+                                    int32_t num_q_heads, const void* q_norm_weight,
+                                    const void* k_norm_weight, const int32_t* positions,
+                                    const int32_t* slot_mapping, float eps, float rope_theta,
+                                    void* q_out, void* k_pool, void* v_pool, pkv_pool_desc pool,
+                                    pkv_stream_t stream);
+
+/*
+ * pkv_kv_append_cow -- append new K/V rows to page tables that may share
+ * pages (a common prompt prefix), copying a shared page before writing into
+ * it (mini-vllm advanced series design, Phase C, adv05 "Radix Attention +
+ * Copy-on-Write"; the main series' hash + ref_count).
+ *
+ *   k_new, v_new   [num_tokens][Hkv][d] bf16
+ *   token_req      [num_tokens] int32: the request (row of page_table) of
+ *                  each new row; a request's rows contiguous and in
+ *                  increasing position
+ *   token_pos      [num_tokens] int32: the row's position in its request
+ *   page_table     [batch][max_pages] int32, UPDATED: an entry whose page
+ *                  is copied is pointed at the copy
+ *   page_refcount  [num_pages] int32, UPDATED: how many table entries name
+ *                  each page
+ *   free_pages     [num_free] int32: pages the call may take, in order
+ *   free_used      one int32 (device): the caller sets it (usually to 0);
+ *                  the call adds the number of pages it took, which are
+ *                  free_pages[old value ..] in some order of requests
+ *
+ * The page holding a request's first new row, and each page a new row
+ * starts at offset 0, is settled first: if no other table entry names it,
+ * the rows go in place; otherwise the request takes the next free page,
+ * rows 0 .. offset-1 of the shared page (every KV head, K and V) are copied
+ * into it, its table entry and counts are updated, and the new rows go
+ * there.  Which sharer keeps the page and which free page each request gets
+ * depend on timing; what each request reads through its table does not.
+ * Pages opened by the new rows must already be in the tables (count 1).
+ * An exhausted free list raises PKV_FLAG_NO_FREE_PAGE and sets the entry to
+ * -1 (its rows are skipped).  Two kernels, the second launched as a
+ * programmatic dependent of the first.
+ */
+PKV_API int pkv_kv_append_cow(const void* k_new, const void* v_new, const int32_t* token_req,
+                              const int32_t* token_pos, int32_t num_tokens, int32_t* page_table,
+                              int32_t batch, int32_t max_pages, int32_t* page_refcount,
+                              const int32_t* free_pages, int32_t num_free, int32_t* free_used,
+                              void* k_pool, void* v_pool, pkv_pool_desc pool, pkv_stream_t stream);
 
 /* Human-readable name of a pkv_status value (static string). */
 PKV_API const char* pkv_status_string(int status);

@@ -27,7 +27,7 @@ __all__ = [
     "PkvError", "LIB_PATH", "pool_desc", "pkv_kv_append", "pkv_decode_workspace_bytes",
     "pkv_paged_attn_decode", "pkv_split_k_combine", "pkv_paged_attn_chunked_prefill",
     "pkv_status_string", "pkv_device_error_flags", "decode_workspace",
-    "pkv_paged_attn_decode_static",
+    "pkv_paged_attn_decode_static", "pkv_qk_norm_rope_append", "pkv_kv_append_cow",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -38,6 +38,7 @@ FLAG_BAD_SLOT = 0x4
 FLAG_BAD_QUERY_ROWS = 0x8
 FLAG_BAD_PAGE = 0x10
 FLAG_INTERNAL = 0x20
+FLAG_NO_FREE_PAGE = 0x40
 
 
 class PkvError(RuntimeError):
@@ -73,6 +74,10 @@ def _load() -> ctypes.CDLL:
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_device_error_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
     lib.pkv_device_error_flags.restype = ctypes.c_int
+    lib.pkv_qk_norm_rope_append.argtypes = [P, P, P, I32, I32, P, P, P, P, F32, F32, P, P, P, _PoolDesc, P]
+    lib.pkv_qk_norm_rope_append.restype = ctypes.c_int
+    lib.pkv_kv_append_cow.argtypes = [P, P, P, P, I32, P, I32, I32, P, P, I32, P, P, P, _PoolDesc, P]
+    lib.pkv_kv_append_cow.restype = ctypes.c_int
     return lib
 
 
@@ -223,6 +228,59 @@ def pkv_paged_attn_chunked_prefill(q, cu_q_lens, ctx_offsets, k_pool, v_pool, pa
         _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table), page_table.shape[1],
         float(scale), _ptr(out), _stream(stream)))
     return out
+
+
+def pkv_qk_norm_rope_append(q, k, v, q_norm_weight, k_norm_weight, positions, slot_mapping, k_pool,
+                            v_pool, eps=1e-6, rope_theta=1e6, q_out=None, stream=None):
+    """RMSNorm + RoPE of this step's q [T, Hq, d] and k [T, Hkv, d] rows, and
+    the write of k (rotated) and v into the pool slots; returns q_out."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 3)
+    for t, n in ((q_norm_weight, "q_norm_weight"), (k_norm_weight, "k_norm_weight")):
+        _need(t, n, torch.bfloat16, 1)
+    _need(positions, "positions", torch.int32, 1)
+    _need(slot_mapping, "slot_mapping", torch.int32, 1)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    T, hq, d = q.shape
+    if k.shape != v.shape or k.shape[0] != T or positions.shape[0] != T or slot_mapping.shape[0] != T:
+        raise ValueError("q, k, v, positions and slot_mapping disagree on the token count")
+    if k.shape[1:] != (k_pool.shape[1], k_pool.shape[3]) or v_pool.shape != k_pool.shape:
+        raise ValueError("row shape does not match the pool")
+    if q_norm_weight.shape[0] != d or k_norm_weight.shape[0] != d or q.shape[2] != d:
+        raise ValueError("norm weights must have head_dim elements")
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    _need(q_out, "q_out", torch.bfloat16, 3)
+    _check("pkv_qk_norm_rope_append", _lib.pkv_qk_norm_rope_append(
+        _ptr(q), _ptr(k), _ptr(v), T, hq, _ptr(q_norm_weight), _ptr(k_norm_weight), _ptr(positions),
+        _ptr(slot_mapping), float(eps), float(rope_theta), _ptr(q_out), _ptr(k_pool), _ptr(v_pool),
+        pool_desc(k_pool), _stream(stream)))
+    return q_out
+
+
+def pkv_kv_append_cow(k_new, v_new, token_req, token_pos, page_table, page_refcount, free_pages,
+                      free_used, k_pool, v_pool, stream=None):
+    """Append rows k_new/v_new [T, Hkv, d] at (token_req, token_pos), copying
+    shared pages first; updates page_table, page_refcount and free_used."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _need(t, n, torch.bfloat16, 3)
+    for t, n in ((token_req, "token_req"), (token_pos, "token_pos"), (page_refcount, "page_refcount"),
+                 (free_pages, "free_pages"), (free_used, "free_used")):
+        _need(t, n, torch.int32, 1)
+    _need(page_table, "page_table", torch.int32, 2)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    T = k_new.shape[0]
+    if v_new.shape != k_new.shape or token_req.shape[0] != T or token_pos.shape[0] != T:
+        raise ValueError("k_new, v_new, token_req and token_pos disagree on the token count")
+    if page_refcount.shape[0] != k_pool.shape[0] or v_pool.shape != k_pool.shape:
+        raise ValueError("page_refcount must have one count per pool page")
+    _check("pkv_kv_append_cow", _lib.pkv_kv_append_cow(
+        _ptr(k_new), _ptr(v_new), _ptr(token_req), _ptr(token_pos), T, _ptr(page_table),
+        page_table.shape[0], page_table.shape[1], _ptr(page_refcount), _ptr(free_pages),
+        free_pages.shape[0], _ptr(free_used), _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool),
+        _stream(stream)))
 
 
 # ------------------------------------------------ decode with built-in scratch

@@ -10,9 +10,11 @@
 #include <mutex>
 #include <unordered_map>
 
+#include "cow.cuh"
 #include "decode.cuh"
 #include "kv_append.cuh"
 #include "prefill.cuh"
+#include "prologue.cuh"
 
 namespace {
 
@@ -530,6 +532,98 @@ int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int3
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if (D == 128) return dispatch_prefill_group<128>(group, prm, qmap, kmap, vmap, max_q_len, s);
   return dispatch_prefill_group<64>(group, prm, qmap, kmap, vmap, max_q_len, s);
+}
+
+int pkv_qk_norm_rope_append(const void* q, const void* k, const void* v, int32_t num_tokens,
+                            int32_t num_q_heads, const void* q_norm_weight, const void* k_norm_weight,
+                            const int32_t* positions, const int32_t* slot_mapping, float eps,
+                            float rope_theta, void* q_out, void* k_pool, void* v_pool, pkv_pool_desc pool,
+                            pkv_stream_t stream) {
+  if (num_tokens < 0) return PKV_ERR_BAD_SHAPE;
+  int st = check_pool(pool);
+  if (st != PKV_OK) return st;
+  int group = 0;
+  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
+  if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(rope_theta) || !(rope_theta > 1.f))
+    return PKV_ERR_BAD_SHAPE;
+  if (num_tokens == 0) return PKV_OK;
+  if (!q || !k || !v || !q_norm_weight || !k_norm_weight || !positions || !slot_mapping || !q_out ||
+      !k_pool || !v_pool)
+    return PKV_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_norm_weight) ||
+      !aligned16(k_norm_weight) || !aligned16(q_out) || !aligned16(k_pool) || !aligned16(v_pool))
+    return PKV_ERR_MISALIGNED;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  pkv::prologue::Params prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.k = static_cast<const uint16_t*>(k);
+  prm.v = static_cast<const uint16_t*>(v);
+  prm.q_w = static_cast<const uint16_t*>(q_norm_weight);
+  prm.k_w = static_cast<const uint16_t*>(k_norm_weight);
+  prm.positions = positions;
+  prm.slots = slot_mapping;
+  prm.q_out = static_cast<uint16_t*>(q_out);
+  prm.k_pool = static_cast<uint16_t*>(k_pool);
+  prm.v_pool = static_cast<uint16_t*>(v_pool);
+  prm.T = num_tokens;
+  prm.Hq = num_q_heads;
+  prm.Hkv = pool.num_kv_heads;
+  prm.P = pool.page_size;
+  prm.num_slots = static_cast<int64_t>(pool.num_pages) * pool.page_size;
+  prm.eps = eps;
+  prm.log2_theta = std::log2(static_cast<double>(rope_theta));
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(static_cast<unsigned>(num_tokens)), block(32 * pkv::prologue::kWarps);
+  if (pool.head_dim == 128) return launch_pdl(pkv::prologue::qk_norm_rope_append_kernel<128>, grid, block, 0, s, prm);
+  return launch_pdl(pkv::prologue::qk_norm_rope_append_kernel<64>, grid, block, 0, s, prm);
+}
+
+int pkv_kv_append_cow(const void* k_new, const void* v_new, const int32_t* token_req, const int32_t* token_pos,
+                      int32_t num_tokens, int32_t* page_table, int32_t batch, int32_t max_pages,
+                      int32_t* page_refcount, const int32_t* free_pages, int32_t num_free, int32_t* free_used,
+                      void* k_pool, void* v_pool, pkv_pool_desc pool, pkv_stream_t stream) {
+  if (num_tokens < 0 || batch < 0 || max_pages <= 0 || num_free < 0) return PKV_ERR_BAD_SHAPE;
+  int st = check_pool(pool);
+  if (st != PKV_OK) return st;
+  if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k_new || !v_new || !token_req || !token_pos || !page_table || !page_refcount || !free_used ||
+      !k_pool || !v_pool || (num_free > 0 && !free_pages))
+    return PKV_ERR_NULL_POINTER;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+    return PKV_ERR_MISALIGNED;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  pkv::cow::Params prm;
+  prm.k_new = static_cast<const uint4*>(k_new);
+  prm.v_new = static_cast<const uint4*>(v_new);
+  prm.token_req = token_req;
+  prm.token_pos = token_pos;
+  prm.page_table = page_table;
+  prm.refcount = page_refcount;
+  prm.free_pages = free_pages;
+  prm.free_used = free_used;
+  prm.k_pool = static_cast<uint4*>(k_pool);
+  prm.v_pool = static_cast<uint4*>(v_pool);
+  prm.T = num_tokens;
+  prm.B = batch;
+  prm.max_pages = max_pages;
+  prm.num_free = num_free;
+  prm.num_pages = pool.num_pages;
+  prm.Hkv = pool.num_kv_heads;
+  prm.P = pool.page_size;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 pgrid(static_cast<unsigned>((num_tokens + pkv::cow::kPrepWarps - 1) / pkv::cow::kPrepWarps));
+  const dim3 pblock(32 * pkv::cow::kPrepWarps);
+  const long long chunks = static_cast<long long>(num_tokens) * pool.num_kv_heads * (pool.head_dim / 8);
+  const unsigned ablocks = static_cast<unsigned>(std::min<long long>((chunks + 255) / 256, dev.sm_count * 16ll));
+  if (pool.head_dim == 128) {
+    if ((st = launch_pdl(pkv::cow::prepare_kernel<128>, pgrid, pblock, 0, s, prm)) != PKV_OK) return st;
+    return launch_pdl(pkv::cow::append_kernel<128>, dim3(ablocks), dim3(256), 0, s, prm);
+  }
+  if ((st = launch_pdl(pkv::cow::prepare_kernel<64>, pgrid, pblock, 0, s, prm)) != PKV_OK) return st;
+  return launch_pdl(pkv::cow::append_kernel<64>, dim3(ablocks), dim3(256), 0, s, prm);
 }
 
 int pkv_device_error_flags(uint32_t* flags, int clear) {
