@@ -176,6 +176,27 @@ PKV_API int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_he
                           float* out_lse, pkv_stream_t stream);
 
 /*
+ * pkv_paged_attn_decode_flags -- pkv_paged_attn_decode with option bits
+ * (the pages have no counterpart; a scheduling option of this library):
+ *   PKV_DECODE_METADATA_READY  the kernel just ahead of this call on
+ *               `stream` writes neither kv_lens nor page_table (for instance
+ *               it is pkv_kv_append or another decode, and the tables were
+ *               copied in earlier).  With the automatic split the decode
+ *               kernel then plans, and reads each warp's first page-table
+ *               entries, while that kernel is still finishing; q, the pools
+ *               and the workspace are still read only after it completes.
+ *               Ignored for a fixed partition.
+ * Unknown bits give PKV_ERR_BAD_SHAPE.  flags = 0 is pkv_paged_attn_decode.
+ */
+#define PKV_DECODE_METADATA_READY 1u
+PKV_API int pkv_paged_attn_decode_flags(const void* q, int32_t batch, int32_t num_q_heads,
+                                        const void* k_pool, const void* v_pool, pkv_pool_desc pool,
+                                        const int32_t* page_table, int32_t max_pages,
+                                        const int32_t* kv_lens, float scale, int32_t partition_tokens,
+                                        void* workspace, size_t workspace_bytes, void* out,
+                                        float* out_lse, uint32_t flags, pkv_stream_t stream);
+
+/*
  * pkv_split_k_combine -- merge split-K partials by their log-sum-exp weights
  * (mini-vllm advanced series design, adv04 "Flash-Decoding"; the formula is
  * the plain reading: M = max_s lse_s, w_s = exp(lse_s - M),
@@ -222,6 +243,41 @@ PKV_API int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_le
                                    const void* v_pool, pkv_pool_desc pool,
                                    const int32_t* page_table, int32_t max_pages, float scale,
                                    void* out, pkv_stream_t stream);
+
+/*
+ * pkv_verify_workspace_bytes -- bytes of workspace pkv_paged_attn_verify
+ * needs for total_q chunk rows whose requests hold at most max_kv_len keys
+ * (pass max_pages * page_size); partition_tokens as in the call.
+ */
+PKV_API size_t pkv_verify_workspace_bytes(int32_t total_q, int32_t num_q_heads, int32_t head_dim,
+                                          int32_t max_kv_len, int32_t partition_tokens);
+
+/*
+ * pkv_paged_attn_verify -- causal attention of short query chunks (2 to 16
+ * rows per request, e.g. the draft tokens a speculative decoder verifies)
+ * over long paged contexts, split along the keys (mini-vllm advanced series
+ * design, Phase B: adv03 speculative decoding's verify step and adv04
+ * flash-decoding's split-K; tiny-llm blog, week 3 optional chapter).  The
+ * rows and their masking are those of pkv_paged_attn_chunked_prefill (row i
+ * of request r sits at ctx_offsets[r] + i and sees keys 0 .. ctx_offsets[r]
+ * + i); the keys of each request are cut into partitions of
+ * partition_tokens, each handled by its own CTAs on the tensor cores, and
+ * the partials are merged by pkv_split_k_combine's rule in a second kernel.
+ *
+ *   partition_tokens  0 = automatic (about four partitions per request of
+ *               max_pages * page_size keys, within [512, 4096]), else a
+ *               multiple of 64
+ *   workspace   device scratch of pkv_verify_workspace_bytes(...) bytes,
+ *               256-byte aligned; no zeroing needed (the call clears what it
+ *               needs on `stream`); calls sharing it must not overlap
+ *   other arguments as pkv_paged_attn_chunked_prefill
+ */
+PKV_API int pkv_paged_attn_verify(const void* q, const int32_t* cu_q_lens, int32_t batch,
+                                  int32_t num_q_heads, int32_t total_q, int32_t max_q_len,
+                                  const int32_t* ctx_offsets, const void* k_pool, const void* v_pool,
+                                  pkv_pool_desc pool, const int32_t* page_table, int32_t max_pages,
+                                  float scale, int32_t partition_tokens, void* workspace,
+                                  size_t workspace_bytes, void* out, pkv_stream_t stream);
 
 /*
  * pkv_paged_attn_decode_static -- pkv_paged_attn_decode without a

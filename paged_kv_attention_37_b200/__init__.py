@@ -28,6 +28,8 @@ __all__ = [
     "pkv_paged_attn_decode", "pkv_split_k_combine", "pkv_paged_attn_chunked_prefill",
     "pkv_status_string", "pkv_device_error_flags", "decode_workspace",
     "pkv_paged_attn_decode_static", "pkv_qk_norm_rope_append", "pkv_kv_append_cow",
+    "pkv_verify_workspace_bytes", "verify_workspace", "pkv_paged_attn_verify", "pkv_paged_attn_decode_flags",
+    "DECODE_METADATA_READY",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -39,6 +41,8 @@ FLAG_BAD_QUERY_ROWS = 0x8
 FLAG_BAD_PAGE = 0x10
 FLAG_INTERNAL = 0x20
 FLAG_NO_FREE_PAGE = 0x40
+
+DECODE_METADATA_READY = 0x1  # pkv_paged_attn_decode_flags option bit
 
 
 class PkvError(RuntimeError):
@@ -78,6 +82,14 @@ def _load() -> ctypes.CDLL:
     lib.pkv_qk_norm_rope_append.restype = ctypes.c_int
     lib.pkv_kv_append_cow.argtypes = [P, P, P, P, I32, P, I32, I32, P, P, I32, P, P, P, _PoolDesc, P]
     lib.pkv_kv_append_cow.restype = ctypes.c_int
+    lib.pkv_paged_attn_decode_flags.argtypes = [P, I32, I32, P, P, _PoolDesc, P, I32, P, F32, I32, P, SZ,
+                                                P, P, ctypes.c_uint32, P]
+    lib.pkv_paged_attn_decode_flags.restype = ctypes.c_int
+    lib.pkv_verify_workspace_bytes.argtypes = [I32, I32, I32, I32, I32]
+    lib.pkv_verify_workspace_bytes.restype = SZ
+    lib.pkv_paged_attn_verify.argtypes = [P, P, I32, I32, I32, I32, P, P, P, _PoolDesc, P, I32, F32, I32, P,
+                                          SZ, P, P]
+    lib.pkv_paged_attn_verify.restype = ctypes.c_int
     return lib
 
 
@@ -165,6 +177,14 @@ def pkv_paged_attn_decode(q, k_pool, v_pool, page_table, kv_lens, scale, partiti
     Returns ``out`` (bf16 [B, Hq, d]); fills ``out_lse`` (fp32 [B, Hq]) if given.
     ``workspace`` (uint8, zero-filled before first use) defaults to a new one.
     """
+    return pkv_paged_attn_decode_flags(q, k_pool, v_pool, page_table, kv_lens, scale, partition_tokens,
+                                       workspace, out, out_lse, 0, stream)
+
+
+def pkv_paged_attn_decode_flags(q, k_pool, v_pool, page_table, kv_lens, scale, partition_tokens=0,
+                                workspace=None, out=None, out_lse=None, flags=0, stream=None):
+    """pkv_paged_attn_decode with option bits (DECODE_METADATA_READY: the
+    kernel just ahead on the stream writes neither kv_lens nor page_table)."""
     _need(q, "q", torch.bfloat16, 3)
     _need(k_pool, "k_pool", torch.bfloat16, 4)
     _need(v_pool, "v_pool", torch.bfloat16, 4)
@@ -183,10 +203,10 @@ def pkv_paged_attn_decode(q, k_pool, v_pool, page_table, kv_lens, scale, partiti
     _need(out, "out", torch.bfloat16, 3)
     if out_lse is not None:
         _need(out_lse, "out_lse", torch.float32, 2)
-    _check("pkv_paged_attn_decode", _lib.pkv_paged_attn_decode(
+    _check("pkv_paged_attn_decode_flags", _lib.pkv_paged_attn_decode_flags(
         _ptr(q), B, hq, _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table),
         max_pages, _ptr(kv_lens), float(scale), int(partition_tokens), _ptr(workspace),
-        workspace.numel(), _ptr(out), _ptr(out_lse), _stream(stream)))
+        workspace.numel(), _ptr(out), _ptr(out_lse), int(flags), _stream(stream)))
     return out
 
 
@@ -227,6 +247,44 @@ def pkv_paged_attn_chunked_prefill(q, cu_q_lens, ctx_offsets, k_pool, v_pool, pa
         _ptr(q), _ptr(cu_q_lens), B, hq, total_q, int(max_q_len), _ptr(ctx_offsets),
         _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table), page_table.shape[1],
         float(scale), _ptr(out), _stream(stream)))
+    return out
+
+
+def pkv_verify_workspace_bytes(total_q, num_q_heads, head_dim, max_kv_len, partition_tokens=0) -> int:
+    return int(_lib.pkv_verify_workspace_bytes(total_q, num_q_heads, head_dim, max_kv_len, partition_tokens))
+
+
+def verify_workspace(total_q, num_q_heads, head_dim, max_kv_len, partition_tokens=0, device=None):
+    """A workspace of the size pkv_paged_attn_verify needs (no zeroing needed)."""
+    n = pkv_verify_workspace_bytes(total_q, num_q_heads, head_dim, max_kv_len, partition_tokens)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def pkv_paged_attn_verify(q, cu_q_lens, ctx_offsets, k_pool, v_pool, page_table, scale, max_q_len,
+                          partition_tokens=0, workspace=None, out=None, stream=None):
+    """Causal attention of short chunks q [total_q, Hq, d] at context offsets,
+    split along the keys (speculative verify); same rows as chunked prefill."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(cu_q_lens, "cu_q_lens", torch.int32, 1)
+    _need(ctx_offsets, "ctx_offsets", torch.int32, 1)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    _need(page_table, "page_table", torch.int32, 2)
+    total_q, hq, d = q.shape
+    B = ctx_offsets.shape[0]
+    if cu_q_lens.shape[0] != B + 1 or page_table.shape[0] != B:
+        raise ValueError("cu_q_lens must have B+1 entries and page_table B rows")
+    if workspace is None:
+        workspace = verify_workspace(total_q, hq, d, page_table.shape[1] * k_pool.shape[2],
+                                     partition_tokens, q.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 3)
+    _check("pkv_paged_attn_verify", _lib.pkv_paged_attn_verify(
+        _ptr(q), _ptr(cu_q_lens), B, hq, total_q, int(max_q_len), _ptr(ctx_offsets), _ptr(k_pool),
+        _ptr(v_pool), pool_desc(k_pool), _ptr(page_table), page_table.shape[1], float(scale),
+        int(partition_tokens), _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream)))
     return out
 
 

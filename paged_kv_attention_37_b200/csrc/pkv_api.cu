@@ -279,25 +279,17 @@ int dispatch_decode_group(int group, const pkv::decode::Params& prm, int sm_coun
 }
 
 // ----------------------------------------------------------- prefill launch
-#ifndef PKV_PREFILL_BN
-#define PKV_PREFILL_BN 64
-#endif
-
 template <int D, int G>
 int launch_prefill(const pkv::prefill::Params& prm, const CUtensorMap& qmap, const CUtensorMap& kmap,
                    const CUtensorMap& vmap, int32_t max_q_len, cudaStream_t stream) {
-  constexpr int BN = PKV_PREFILL_BN;  // keys per tile
-  using LY = pkv::prefill::Layout<D, BN>;
-  auto kernel = pkv::prefill::prefill_kernel<D, G, BN>;
-  // BN=64: about half an SM's shared memory, so two CTAs (with 256 TMEM
-  // columns each) share an SM; BN=128: one CTA and 512 columns per SM
-  const size_t smem = BN == 64 ? LY::kBytes : std::max<size_t>(LY::kBytes, 116 * 1024);
+  auto kernel = pkv::prefill::prefill_kernel<D, G, pkv::prefill::kKeyTile>;
+  const size_t smem = pkv::prefill::smem_bytes<D>();
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return PKV_ERR_CUDA;
-  constexpr int QPOS = pkv::prefill::kM / G;
+  constexpr int QPOS = pkv::prefill::kRowsPerCta / G;  // chunk positions per CTA
   const long long tiles = (static_cast<long long>(max_q_len) + QPOS - 1) / QPOS;
-  const long long blocks = tiles * prm.Hkv * prm.B;
+  const long long blocks = tiles * prm.Hkv * prm.B * prm.splits;
   if (blocks == 0) return PKV_OK;
   if (blocks > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
   pkv::prefill::Params args = prm;
@@ -317,6 +309,117 @@ int dispatch_prefill_group(int group, const pkv::prefill::Params& prm, const CUt
     case 8: return launch_prefill<D, 8>(prm, qmap, kmap, vmap, max_q_len, stream);
   }
   return PKV_ERR_UNSUPPORTED;
+}
+
+// Split-K chunk attention (short chunks over long contexts): the automatic
+// partition depends on the longest context only, so the workspace size can
+// be computed without device data: about four splits per request, a
+// multiple of the key tile, within [512, 4096] keys.
+constexpr int kPrefillBN = pkv::prefill::kKeyTile;
+
+int32_t verify_partition(int32_t max_kv_len, int32_t partition_tokens) {
+  if (partition_tokens > 0) return partition_tokens;
+  const int32_t quarter = (std::max<int32_t>(max_kv_len, 1) + 3) / 4;
+  const int32_t part = (quarter + kPrefillBN - 1) / kPrefillBN * kPrefillBN;
+  return std::min<int32_t>(4096, std::max<int32_t>(512, part));
+}
+
+struct VerifyLayout {
+  int32_t partition = 0, splits = 1;
+  size_t num_splits = 0, part_lse = 0, part_o = 0, total = 0;
+};
+
+VerifyLayout verify_layout(int32_t total_q, int32_t Hq, int32_t D, int32_t max_kv_len, int32_t partition_tokens) {
+  VerifyLayout v;
+  v.partition = verify_partition(max_kv_len, partition_tokens);
+  v.splits = std::max<int32_t>(1, (max_kv_len + v.partition - 1) / v.partition);
+  const size_t rows = static_cast<size_t>(total_q) * Hq;
+  v.num_splits = 0;
+  v.part_lse = align256(static_cast<size_t>(total_q) * 4);
+  v.part_o = v.part_lse + align256(rows * v.splits * 4);
+  v.total = v.part_o + align256(rows * v.splits * D * 4);
+  return v;
+}
+
+// Chunked prefill (split_tokens = 0) or its split-K form (split_tokens =
+// the partition, -1 = automatic; workspace as verify_layout).
+int run_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t num_q_heads, int32_t total_q,
+                int32_t max_q_len, const int32_t* ctx_offsets, const void* k_pool, const void* v_pool,
+                const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages, float scale,
+                int32_t split_tokens, void* workspace, size_t workspace_bytes, void* out, cudaStream_t s) {
+  if (batch < 0 || total_q < 0 || max_q_len < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
+  int st = check_pool(pool);
+  if (st != PKV_OK) return st;
+  int group = 0;
+  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return PKV_ERR_BAD_SHAPE;
+  if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
+  if (batch == 0 || total_q == 0 || max_q_len == 0) return PKV_OK;
+  if (!q || !cu_q_lens || !ctx_offsets || !k_pool || !v_pool || !page_table || !out)
+    return PKV_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return PKV_ERR_MISALIGNED;
+  VerifyLayout vl;
+  if (split_tokens != 0) {
+    vl = verify_layout(total_q, num_q_heads, pool.head_dim, max_pages * pool.page_size,
+                       split_tokens < 0 ? 0 : split_tokens);
+    if (workspace == nullptr || workspace_bytes < vl.total) return PKV_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  }
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  const int D = pool.head_dim;
+  const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
+  const int qpos = pkv::prefill::kRowsPerCta / group;
+  CUtensorMap qmap, kmap, vmap;
+  if ((st = make_map(&qmap, q, D, num_q_heads, total_q, D * 2ull, static_cast<uint64_t>(num_q_heads) * D * 2, 64,
+                     group, qpos, true)) != PKV_OK)
+    return st;
+  if ((st = make_map(&kmap, k_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
+                     pool.page_size, 1, true)) != PKV_OK)
+    return st;
+  if ((st = make_map(&vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
+                     pool.page_size, 1, true)) != PKV_OK)
+    return st;
+  pkv::prefill::Params prm;
+  prm.cu_q_lens = cu_q_lens;
+  prm.ctx_offsets = ctx_offsets;
+  prm.page_table = page_table;
+  prm.out = static_cast<uint16_t*>(out);
+  prm.B = batch;
+  prm.Hq = num_q_heads;
+  prm.Hkv = pool.num_kv_heads;
+  prm.P = pool.page_size;
+  prm.max_pages = max_pages;
+  prm.num_pages = pool.num_pages;
+  prm.total_q = total_q;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.partition = 0;
+  prm.splits = 1;
+  prm.part_o = nullptr;
+  prm.part_lse = nullptr;
+  prm.num_splits = nullptr;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (split_tokens != 0) {
+    prm.partition = vl.partition;
+    prm.splits = vl.splits;
+    prm.num_splits = reinterpret_cast<int32_t*>(ws + vl.num_splits);
+    prm.part_lse = reinterpret_cast<float*>(ws + vl.part_lse);
+    prm.part_o = reinterpret_cast<float*>(ws + vl.part_o);
+    // rows the kernel does not reach (past cu_q_lens[batch]) must read as
+    // "one split" to the combine, which then leaves them alone
+    if (cudaMemsetAsync(prm.num_splits, 0, static_cast<size_t>(total_q) * 4, s) != cudaSuccess) return PKV_ERR_CUDA;
+  }
+  st = D == 128 ? dispatch_prefill_group<128>(group, prm, qmap, kmap, vmap, max_q_len, s)
+                : dispatch_prefill_group<64>(group, prm, qmap, kmap, vmap, max_q_len, s);
+  if (st != PKV_OK || split_tokens == 0) return st;
+  // merge the rows whose request was split (rows of single-split requests
+  // were written by the kernel itself)
+  if (D == 128)
+    return launch_combine<128>(prm.part_o, prm.part_lse, prm.num_splits, total_q, num_q_heads, prm.splits,
+                               prm.out, nullptr, 1, true, s);
+  return launch_combine<64>(prm.part_o, prm.part_lse, prm.num_splits, total_q, num_q_heads, prm.splits,
+                            prm.out, nullptr, 1, true, s);
 }
 
 // Host-side checks shared by both decode entry points, and the split and
@@ -362,7 +465,7 @@ int check_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* 
 int run_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool, const void* v_pool,
                const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages,
                const int32_t* kv_lens, float scale, int32_t partition_tokens, const DecodePlan& dp,
-               void* workspace, void* out, float* out_lse, cudaStream_t s) {
+               void* workspace, void* out, float* out_lse, uint32_t flags, cudaStream_t s) {
   DeviceInfo dev;
   int st;
   if ((st = current_device(&dev)) != PKV_OK) return st;
@@ -391,6 +494,7 @@ int run_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_
   prm.partition = partition_tokens;
   prm.merge_nodes = dp.ss.nodes;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.meta_ready = (flags & PKV_DECODE_METADATA_READY) ? 1 : 0;
   if ((st = prepare_workspace(workspace, wl.zero_bytes, s)) != PKV_OK) return st;
   if (pool.head_dim == 128) return dispatch_decode_group<128>(dp.group, prm, dev.sm_count, s);
   return dispatch_decode_group<64>(dp.group, prm, dev.sm_count, s);
@@ -455,6 +559,16 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
                           int32_t max_pages, const int32_t* kv_lens, float scale,
                           int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                           void* out, float* out_lse, pkv_stream_t stream) {
+  return pkv_paged_attn_decode_flags(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens,
+                                     scale, partition_tokens, workspace, workspace_bytes, out, out_lse, 0u, stream);
+}
+
+int pkv_paged_attn_decode_flags(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool,
+                                const void* v_pool, pkv_pool_desc pool, const int32_t* page_table,
+                                int32_t max_pages, const int32_t* kv_lens, float scale,
+                                int32_t partition_tokens, void* workspace, size_t workspace_bytes, void* out,
+                                float* out_lse, uint32_t flags, pkv_stream_t stream) {
+  if ((flags & ~static_cast<uint32_t>(PKV_DECODE_METADATA_READY)) != 0) return PKV_ERR_BAD_SHAPE;
   DecodePlan dp;
   const int st = check_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens,
                               scale, partition_tokens, out, &dp);
@@ -462,7 +576,7 @@ int pkv_paged_attn_decode(const void* q, int32_t batch, int32_t num_q_heads, con
   if (workspace == nullptr || workspace_bytes < dp.wl.total) return PKV_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
   return run_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens, scale,
-                    partition_tokens, dp, workspace, out, out_lse, reinterpret_cast<cudaStream_t>(stream));
+                    partition_tokens, dp, workspace, out, out_lse, flags, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
@@ -489,49 +603,27 @@ int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int3
                                    const int32_t* ctx_offsets, const void* k_pool, const void* v_pool,
                                    pkv_pool_desc pool, const int32_t* page_table, int32_t max_pages,
                                    float scale, void* out, pkv_stream_t stream) {
-  if (batch < 0 || total_q < 0 || max_q_len < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
-  int st = check_pool(pool);
-  if (st != PKV_OK) return st;
-  int group = 0;
-  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
-  if (!std::isfinite(scale) || !(scale > 0.f)) return PKV_ERR_BAD_SHAPE;
-  if (batch == 0 || total_q == 0 || max_q_len == 0) return PKV_OK;
-  if (!q || !cu_q_lens || !ctx_offsets || !k_pool || !v_pool || !page_table || !out)
-    return PKV_ERR_NULL_POINTER;
-  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
-    return PKV_ERR_MISALIGNED;
-  if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != PKV_OK) return st;
-  const int D = pool.head_dim;
-  const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
-  const int qpos = pkv::prefill::kM / group;
-  CUtensorMap qmap, kmap, vmap;
-  if ((st = make_map(&qmap, q, D, num_q_heads, total_q, D * 2ull, static_cast<uint64_t>(num_q_heads) * D * 2, 64,
-                     group, qpos, true)) != PKV_OK)
-    return st;
-  if ((st = make_map(&kmap, k_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
-                     pool.page_size, 1, true)) != PKV_OK)
-    return st;
-  if ((st = make_map(&vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
-                     pool.page_size, 1, true)) != PKV_OK)
-    return st;
-  pkv::prefill::Params prm;
-  prm.cu_q_lens = cu_q_lens;
-  prm.ctx_offsets = ctx_offsets;
-  prm.page_table = page_table;
-  prm.out = static_cast<uint16_t*>(out);
-  prm.B = batch;
-  prm.Hq = num_q_heads;
-  prm.Hkv = pool.num_kv_heads;
-  prm.P = pool.page_size;
-  prm.max_pages = max_pages;
-  prm.num_pages = pool.num_pages;
-  prm.total_q = total_q;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  auto s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 128) return dispatch_prefill_group<128>(group, prm, qmap, kmap, vmap, max_q_len, s);
-  return dispatch_prefill_group<64>(group, prm, qmap, kmap, vmap, max_q_len, s);
+  return run_prefill(q, cu_q_lens, batch, num_q_heads, total_q, max_q_len, ctx_offsets, k_pool, v_pool, pool,
+                     page_table, max_pages, scale, 0, nullptr, 0, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t pkv_verify_workspace_bytes(int32_t total_q, int32_t num_q_heads, int32_t head_dim, int32_t max_kv_len,
+                                  int32_t partition_tokens) {
+  if (total_q < 0 || num_q_heads < 0 || head_dim < 0 || max_kv_len < 0 || partition_tokens < 0) return 0;
+  return verify_layout(total_q, num_q_heads, head_dim, max_kv_len, partition_tokens).total;
+}
+
+int pkv_paged_attn_verify(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t num_q_heads,
+                          int32_t total_q, int32_t max_q_len, const int32_t* ctx_offsets, const void* k_pool,
+                          const void* v_pool, pkv_pool_desc pool, const int32_t* page_table, int32_t max_pages,
+                          float scale, int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                          void* out, pkv_stream_t stream) {
+  if (partition_tokens < 0 || (partition_tokens > 0 && partition_tokens % kPrefillBN != 0) ||
+      partition_tokens > (1 << 20))
+    return PKV_ERR_BAD_SHAPE;
+  return run_prefill(q, cu_q_lens, batch, num_q_heads, total_q, max_q_len, ctx_offsets, k_pool, v_pool, pool,
+                     page_table, max_pages, scale, partition_tokens == 0 ? -1 : partition_tokens, workspace,
+                     workspace_bytes, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int pkv_qk_norm_rope_append(const void* q, const void* k, const void* v, int32_t num_tokens,
@@ -707,5 +799,5 @@ extern "C" int pkv_paged_attn_decode_static(const void* q, int32_t batch, int32_
   if (cudaMemsetAsync(scratch, 0, dp.wl.zero_bytes, s) != cudaSuccess) return PKV_ERR_CUDA;
   mark_workspace_zero(scratch, dp.wl.zero_bytes);
   return run_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens, scale,
-                    partition_tokens, dp, scratch, out, out_lse, s);
+                    partition_tokens, dp, scratch, out, out_lse, 0u, s);
 }

@@ -14,9 +14,11 @@
 //   S = Q K^T   : M=128, N=BN, K=d  -> TMEM (two buffers, double-buffered)
 //   softmax     : one thread per TMEM lane (= one query row), log2 domain,
 //                 lazy rescale of O only when the running max grows by > 2^8
-//   O += P V    : M=128, N=d, K=BN; P (bf16) staged in shared memory,
-//                 V used as an MN-major operand straight from its tile
-// With BN=64 a CTA needs ~112 KB of shared memory and 256 TMEM columns, so
+//   O += P V    : M=128, N=d, K=BN; P (bf16) written back into tensor memory
+//                 over the S columns it came from and read by the MMA from
+//                 there (A operand in TMEM); V is an MN-major operand
+//                 straight from its tile
+// With BN=64 a CTA needs ~96 KB of shared memory and 256 TMEM columns, so
 // two CTAs share an SM and one CTA's softmax overlaps the other's MMAs.
 // Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer (one
 // thread), warps 2..5 softmax and epilogue.
@@ -29,6 +31,11 @@ namespace prefill {
 
 constexpr int kM = 128;  // query rows per CTA
 constexpr int kThreads = 192;
+// What the launcher needs to know: query rows (positions x group heads) per
+// CTA, keys per K/V tile (split partitions are multiples of it), and the
+// dynamic shared memory of a CTA.
+constexpr int kRowsPerCta = kM;
+constexpr int kKeyTile = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 256x
 
 struct Params {
@@ -39,6 +46,15 @@ struct Params {
   int32_t B, Hq, Hkv, P, max_pages, num_pages, total_q;
   int32_t qtiles;  // query tiles per request in the grid (ceil(max_q_len / rows per tile))
   float scale_log2;
+  // split-K over the keys (short chunks over long contexts): a CTA takes the
+  // keys [s*partition, (s+1)*partition) of its request and, when the request
+  // has more than one split, writes a partial normalised within the split and
+  // its lse for the combine kernel.  partition = 0: no split (splits = 1).
+  int32_t partition;    // keys per split, a multiple of the key tile
+  int32_t splits;       // splits per request in the grid
+  float* part_o;        // [total_q][Hq][splits][D]
+  float* part_lse;      // [total_q][Hq][splits]
+  int32_t* num_splits;  // [total_q]: splits of each chunk row's request
 };
 
 #ifndef PKV_PREFILL_ORDER
@@ -53,18 +69,20 @@ struct Layout {
   static constexpr int kKVTile = (D / 64) * kKVHalf;    // [D/64][BN rows][128 B]
   static constexpr int kKOff = kQOff + (D / 64) * kQHalf;  // 2 stages
   static constexpr int kVOff = kKOff + 2 * kKVTile;
-  static constexpr int kPOff = kVOff + 2 * kKVTile;     // [BN/64][128 rows][128 B]
-  static constexpr int kBarOff = kPOff + (BN / 64) * kQHalf;
+  static constexpr int kBarOff = kVOff + 2 * kKVTile;   // P lives in TMEM, over its S columns
   static constexpr int kTmemCols = 2 * BN + D <= 256 ? 256 : 512;  // S0, S1, O
   static constexpr int kColS0 = 0, kColS1 = BN, kColO = 2 * BN;
-  // barriers: q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull, pvdone, final, sfree[2]
+  // barriers: q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], pvdone[2], final
   static constexpr int kNumBars = 16;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr size_t kBytes = kTmemSlotOff + 16;  // the base is 1024-byte aligned
 };
 
+template <int D>
+constexpr size_t smem_bytes();
+
 enum Bar { kQ = 0, kKFull = 1, kKEmpty = 3, kVFull = 5, kVEmpty = 7, kSFull = 9, kPFull = 11,
-           kPVDone = 12, kFinal = 13, kSFree = 14 };
+           kPVDone = 13, kFinal = 15 };
 
 template <int D, int G, int BN>
 __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
@@ -87,14 +105,16 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
   // together and share them through L2.  Order 0: heaviest tiles of every
   // request first.
   int r, g, qt_rev;
+  const int split = blockIdx.x % p.splits;  // the splits of a query tile are adjacent
+  const int bx = blockIdx.x / p.splits;
   if (PKV_PREFILL_ORDER == 1) {
-    qt_rev = blockIdx.x % p.qtiles;
-    const int rest = blockIdx.x / p.qtiles;
+    qt_rev = bx % p.qtiles;
+    const int rest = bx / p.qtiles;
     g = rest % p.Hkv;
     r = rest / p.Hkv;
   } else {
-    r = blockIdx.x % p.B;
-    const int rest = blockIdx.x / p.B;
+    r = bx % p.B;
+    const int rest = bx / p.B;
     g = rest % p.Hkv;
     qt_rev = rest / p.Hkv;
   }
@@ -120,7 +140,14 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
   const int pos_lo = c + qt * QPOS;                      // smallest query position in the tile
   const int rows_valid = min(QPOS, n_r - qt * QPOS);     // chunk positions present
   const int kv_end = pos_lo + rows_valid;                // keys 0 .. kv_end-1 are used
-  const int nt = (kv_end + kN - 1) / kN;                 // key tiles
+  // this CTA's key tiles [j0, j0 + nt): all of them, or its split's
+  const bool split_mode = p.partition > 0;
+  const int req_splits = split_mode ? (c + n_r + p.partition - 1) / p.partition : 1;
+  if (split >= req_splits) return;
+  const int j0 = split_mode ? split * (p.partition / kN) : 0;
+  const int j1 = split_mode ? min((kv_end + kN - 1) / kN, j0 + p.partition / kN) : (kv_end + kN - 1) / kN;
+  const int nt = max(0, j1 - j0);                        // key tiles of this CTA
+  const bool to_partial = req_splits > 1;
 
   // 128-byte swizzle atoms need 1024-byte alignment; the declaration asks
   // for it, and a misaligned base (never expected) is refused, not used
@@ -143,10 +170,9 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       mbar_init(bar(kVFull + i), 1);
       mbar_init(bar(kVEmpty + i), 1);
       mbar_init(bar(kSFull + i), 1);
-      mbar_init(bar(kSFree + i), 128);
+      mbar_init(bar(kPFull + i), 128);
+      mbar_init(bar(kPVDone + i), 1);
     }
-    mbar_init(bar(kPFull), 128);
-    mbar_init(bar(kPVDone), 1);
     mbar_init(bar(kFinal), 1);
     fence_barrier_init();
   }
@@ -159,7 +185,6 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
   const uint32_t sQ = sbase + LY::kQOff;
   auto sK = [&](int b) { return sbase + LY::kKOff + b * LY::kKVTile; };
   auto sV = [&](int b) { return sbase + LY::kVOff + b * LY::kKVTile; };
-  const uint32_t sP = sbase + LY::kPOff;
 
   if (warp == 0) {
     // ============================ TMA producer ============================
@@ -179,10 +204,11 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     // page ids of tile j: the request's page-table entries are read 32 at a
     // time, the next 32 already in flight, so no TMA issue waits on them
     const int total_pages = (kv_end + p.P - 1) / p.P;
-    int pid_base = 0;
-    int pid_cur = lane < total_pages ? __ldg(ptab + lane) : -1;
-    int pid_next = 32 + lane < total_pages ? __ldg(ptab + 32 + lane) : -1;
-    auto tile_pages = [&](int j) {
+    int pid_base = (j0 * kN / p.P) & ~31;  // the 32-entry window of the first page
+    int pid_cur = pid_base + lane < total_pages ? __ldg(ptab + pid_base + lane) : -1;
+    int pid_next = pid_base + 32 + lane < total_pages ? __ldg(ptab + pid_base + 32 + lane) : -1;
+    auto tile_pages = [&](int jl) {  // jl: the CTA's local tile index
+      const int j = j0 + jl;
       const int first = j * kN / p.P;
       const int npg = (min(kN, kv_end - j * kN) + p.P - 1) / p.P;
       while (first >= pid_base + 32) {
@@ -244,11 +270,12 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       if (lane == 0) {
 #pragma unroll
         for (int ks = 0; ks < kN / 16; ++ks) {
-          const uint64_t a = smem_desc_sw128(sP + (ks >> 2) * LY::kQHalf + (ks & 3) * 32, 16, 1024);
+          // A = P(i) from TMEM: 16 bf16 per row = 8 columns of its S buffer
+          const uint32_t a = tmem + (b ? kColS1 : kColS0) + ks * 8;
           const uint64_t bdesc = smem_desc_sw128(sV(b) + ks * 16 * 128, LY::kKVHalf, 1024);
-          tc_mma_ss(tmem + kColO, a, bdesc, kIdescPV, i > 0 || ks > 0);
+          tc_mma_ts(tmem + kColO, a, bdesc, kIdescPV, i > 0 || ks > 0);
         }
-        tc_commit(bar(kPVDone));
+        tc_commit(bar(kPVDone + b));
         tc_commit(bar(kVEmpty + b));
       }
       __syncwarp();
@@ -277,11 +304,12 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     while (ok && npv < nt) {
       int act = 0;  // 1: P.V(npv), 2: S(ns); decided by lane 0 for the whole warp
       if (lane == 0) {
-        if (mbar_try_wait(bar(kPFull), npv & 1) && mbar_try_wait(bar(kVFull + (npv & 1)), (npv >> 1) & 1))
+        if (mbar_try_wait(bar(kPFull + (npv & 1)), (npv >> 1) & 1) &&
+            mbar_try_wait(bar(kVFull + (npv & 1)), (npv >> 1) & 1))
           act = 1;
-        else if (ns < nt && mbar_try_wait(bar(kSFree + (ns & 1)), ((ns - 2) >> 1) & 1) &&
+        else if (ns < nt && mbar_try_wait(bar(kPVDone + (ns & 1)), ((ns - 2) >> 1) & 1) &&
                  mbar_try_wait(bar(kKFull + (ns & 1)), (ns >> 1) & 1))
-          act = 2;
+          act = 2;  // S(ns) overwrites the buffer whose P fed PV(ns-2): wait for it
       }
       act = __shfl_sync(0xffffffffu, act, 0);
       if (act == 1) {
@@ -320,14 +348,12 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 #pragma unroll
         for (int cc = 0; cc < kN / 32; ++cc) tmem_ld_32x32b_x32(trow + (b ? kColS1 : kColS0) + cc * 32, v[cc]);
         tmem_wait_ld();
-        tc_fence_before_sync();
-        mbar_arrive(bar(kSFree + b));  // this S buffer may take the next-but-one tile
 #pragma unroll
         for (int cc = 0; cc < kN / 32; ++cc)
 #pragma unroll
           for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(v[cc][e]);
       }
-      const int key0 = j * kN;
+      const int key0 = (j0 + j) * kN;
       if (key0 + kN - 1 > pos_lo || key0 + kN > kv_end) {  // diagonal or ragged tile
 #pragma unroll
         for (int e = 0; e < kN; ++e) {
@@ -345,22 +371,24 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
         alpha = fast_exp2(m - mc);
         m = mc;
       }
-      // p = 2^(s*scale*log2e - m): one FMA and one exp2 per element
+      // p = 2^(s*scale*log2e - m): one FMA and one exp2 per element.  A row
+      // that has seen no visible key yet (possible inside a later split) keeps
+      // m = -inf; its weights are then 2^-inf = 0, never 2^(-inf + inf).
+      const float msub = m == -INFINITY ? 0.f : m;
       uint32_t pk[kN / 2];
       float2 rs = make_float2(0.f, 0.f);
 #pragma unroll
       for (int e = 0; e < kN; e += 2) {
-        const float a0 = fast_exp2(fmaf(s[e], sl2, -m)), a1 = fast_exp2(fmaf(s[e + 1], sl2, -m));
+        const float a0 = fast_exp2(fmaf(s[e], sl2, -msub)), a1 = fast_exp2(fmaf(s[e + 1], sl2, -msub));
         rs = __fadd2_rn(rs, make_float2(a0, a1));
         pk[e / 2] = pack_bf16x2(a0, a1);
       }
       l = fmaf(l, alpha, rs.x + rs.y);
-      if (j >= 1) {
-        // PV of the previous tile must be done: P is single-buffered and O
-        // may need rescaling.
-        if (!mbar_wait(bar(kPVDone), (j - 1) & 1)) { ok = false; break; }
+      if (j >= 1 && __any_sync(0xffffffffu, need)) {
+        // O is rescaled only after PV of the previous tile is done
+        if (!mbar_wait(bar(kPVDone + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, need)) {
+        {
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t v[32];
@@ -373,14 +401,16 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
           tmem_wait_st();
         }
       }
-      // P row -> shared memory, 128-byte swizzle (K-major A operand)
-      uint8_t* prow = smem + LY::kPOff + row * 128;
+      // P row -> TMEM over this tile's S columns (read above), the K-major
+      // A operand of the PV MMA: two bf16 per 32-bit column
 #pragma unroll
-      for (int ch = 0; ch < kN / 8; ++ch) {
-        const int half = ch >> 3, c16 = ch & 7;
-        *reinterpret_cast<uint4*>(prow + half * LY::kQHalf + ((c16 ^ (row & 7)) << 4)) =
-            make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+      for (int cc = 0; cc < kN / 64; ++cc) {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = pk[cc * 32 + e];
+        tmem_st_32x32b_x32(trow + (b ? kColS1 : kColS0) + cc * 32, w);
       }
+      tmem_wait_st();
       if (key0 + kN > kv_end) {
         // ragged last tile: V rows past kv_end were not loaded (or hold
         // unused slots); zero them so 0 * garbage cannot reach O
@@ -395,12 +425,39 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       }
       fence_proxy_async_smem();
       tc_fence_before_sync();
-      mbar_arrive(bar(kPFull));
+      mbar_arrive(bar(kPFull + b));
     }
-    if (ok && nt >= 1 && mbar_wait(bar(kPVDone), (nt - 1) & 1)) {
-      tc_fence_after_sync();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint16_t* dst = p.out + (static_cast<size_t>(q0 + qt * QPOS + pos_local) * p.Hq + g * G + hh) * D;
+    const bool have_o = ok && nt >= 1 && mbar_wait(bar(kPVDone + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1);
+    const size_t qrow = static_cast<size_t>(q0 + qt * QPOS + pos_local);  // this thread's chunk row
+    if (split_mode && split == 0 && g == 0 && hh == 0 && row_valid) p.num_splits[qrow] = req_splits;
+    if (have_o) tc_fence_after_sync();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    if (to_partial && (have_o || (ok && nt == 0))) {
+      // a partial normalised within this split (zero, lse -inf, when the
+      // split holds none of the tile's keys), for the combine kernel
+      const size_t prow = (qrow * p.Hq + g * G + hh) * p.splits + split;
+      float* dst = p.part_o + prow * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        if (have_o) {
+          tmem_ld_32x32b_x32(trow + kColO + cc * 32, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (row_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + cc * 32 + e) =
+                make_float4(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv,
+                            __uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
+        }
+      }
+      if (row_valid) p.part_lse[prow] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    } else if (!to_partial && have_o) {
+      uint16_t* dst = p.out + (qrow * p.Hq + g * G + hh) * D;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
@@ -429,6 +486,11 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+template <int D>
+constexpr size_t smem_bytes() {
+  return Layout<D, kKeyTile>::kBytes;  // about half an SM: two CTAs share one
 }
 
 }  // namespace prefill

@@ -146,6 +146,38 @@ def test_host_validation_without_gpu(lib):
     # a partition below -1 is not one of the documented values
     assert dec(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, -5, ws, 1 << 20, dummy, None, None) == -2
 
+    lib.pkv_paged_attn_decode_flags.argtypes = [P, I32, I32, P, P, PoolDesc, P, I32, P, ctypes.c_float,
+                                                I32, P, ctypes.c_size_t, P, P, ctypes.c_uint32, P]
+    decf = lib.pkv_paged_attn_decode_flags
+    assert decf(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, ws, 1 << 20, dummy, None, 2, None) == -2
+    assert decf(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, ws, 64, dummy, None, 1, None) == -5
+
+    lib.pkv_paged_attn_verify.argtypes = [P, P, I32, I32, I32, I32, P, P, P, PoolDesc, P, I32, ctypes.c_float,
+                                          I32, P, ctypes.c_size_t, P, P]
+    ver = lib.pkv_paged_attn_verify
+    # partition not a multiple of the 64-key tile; workspace missing
+    assert ver(dummy, dummy, 2, 32, 8, 4, dummy, dummy, dummy, good, dummy, 8, 0.1, 100, ws, 1 << 20, dummy, None) == -2
+    assert ver(dummy, dummy, 2, 32, 8, 4, dummy, dummy, dummy, good, dummy, 8, 0.1, 0, None, 0, dummy, None) == -5
+    lib.pkv_verify_workspace_bytes.restype = ctypes.c_size_t
+    lib.pkv_verify_workspace_bytes.argtypes = [I32] * 5
+    # rows x heads x splits partials of d fp32 and their lse, about four splits
+    assert lib.pkv_verify_workspace_bytes(256, 32, 128, 4096, 0) >= 256 * 32 * 4 * 129 * 4
+    assert lib.pkv_verify_workspace_bytes(-1, 32, 128, 4096, 0) == 0
+
+    lib.pkv_qk_norm_rope_append.argtypes = [P, P, P, I32, I32, P, P, P, P, ctypes.c_float, ctypes.c_float,
+                                            P, P, P, PoolDesc, P]
+    pro = lib.pkv_qk_norm_rope_append
+    assert pro(dummy, dummy, dummy, 4, 32, dummy, dummy, dummy, dummy, 1e-6, 1e6, dummy, dummy, dummy, good, None) != -1
+    assert pro(dummy, dummy, dummy, 4, 32, dummy, dummy, dummy, dummy, 1e-6, 0.5, dummy, dummy, dummy, good, None) == -2
+    assert pro(dummy, dummy, dummy, 4, 12, dummy, dummy, dummy, dummy, 1e-6, 1e6, dummy, dummy, dummy, good, None) == -2
+    assert pro(None, dummy, dummy, 4, 32, dummy, dummy, dummy, dummy, 1e-6, 1e6, dummy, dummy, dummy, good, None) == -1
+
+    lib.pkv_kv_append_cow.argtypes = [P, P, P, P, I32, P, I32, I32, P, P, I32, P, P, P, PoolDesc, P]
+    cow = lib.pkv_kv_append_cow
+    assert cow(dummy, dummy, dummy, dummy, 4, dummy, 2, 0, dummy, dummy, 3, dummy, dummy, dummy, good, None) == -2
+    assert cow(dummy, dummy, dummy, dummy, 4, None, 2, 8, dummy, dummy, 3, dummy, dummy, dummy, good, None) == -1
+    assert cow(None, None, None, None, 0, None, 2, 8, None, None, 0, None, None, None, good, None) == 0
+
     lib.pkv_paged_attn_chunked_prefill.argtypes = [P, P, I32, I32, I32, I32, P, P, P, PoolDesc, P,
                                                    I32, ctypes.c_float, P, P]
     pre = lib.pkv_paged_attn_chunked_prefill
