@@ -143,6 +143,7 @@ struct Params {
   uint32_t* group_done;       // [B*Hkv][merge_nodes] finished children per merge node (automatic split)
   int32_t B, Hq, Hkv, P, max_pages, num_pages, S_max, partition, merge_nodes;
   float scale_log2;           // softmax scale * log2(e)
+  int32_t meta_ready;         // the kernel ahead writes neither kv_lens nor page_table
 };
 
 struct ChunkInfo {
@@ -397,8 +398,13 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   static_assert((T == 8 || T == 16) && (D == 64 || D == 128), "head_dim 64 or 128");
   static_assert(NS >= 2, "at least two stages per warp");
   // launched as a programmatic dependent: nothing global is read before the
-  // kernel ahead of it on the stream (usually the append) has completed
-  pdl_wait();
+  // kernel ahead of it on the stream (usually the append) has completed --
+  // except, when the caller vouches that the kernel ahead writes neither the
+  // lengths nor the page table (meta_ready) and the split is automatic (the
+  // plan then reads no workspace counter), the plan and each warp's first
+  // page-table fetch, which so overlap the tail of that kernel
+  const bool early = p.meta_ready != 0 && p.partition == 0;
+  if (!early) pdl_wait();
 
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -692,6 +698,10 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
     return true;
   };
 
+  if (early) {
+    if (more && !active) fetch();
+    pdl_wait();  // the queries, the pools and the workspace come after the kernel ahead
+  }
   // ================================ compute side ================================
   // Score phase: token group tg (token tg of each step); this lane holds E
   // elements of d as E/8 pieces of 8, piece j at elements [8*(T*j + ei), +8).

@@ -213,6 +213,33 @@ def test_decode_workspace_survives_batch_growth(pkv):
     check_no_flags(pkv)
 
 
+@pytest.mark.parametrize("name,over", [
+    ("tiny_decode", {}),
+    ("qwen3_decode", dict(B=8, len_lo=100, len_hi=1100)),
+    ("qwen3_decode", dict(lens=[1, 2, 15, 16, 17, 31, 32, 33, 255, 256, 257])),
+    ("splitk_long", dict(lens=[4000, 8192 + 13, 20000, 33])),
+    ("frag_large", dict(B=24, median=300.0, max_len=2000)),
+    ("qwen3_decode", dict(B=5, len_lo=20, len_hi=700, num_kv_heads=4, num_q_heads=32, head_dim=64)),
+])
+def test_decode_metadata_ready(pkv, name, over):
+    # the plan and first page-table reads run before the wait on the kernel
+    # ahead (here the append, launched just before): same results
+    w = make_workload(name, 13, **over)
+    ds, os_ = DeviceStep(pkv, w), OracleStep(w)
+    os_.append()
+    ref, ref_lse, sel = os_.decode()
+    dec = list(w.decode_ids)
+    ws = pkv.decode_workspace(len(dec), w.num_q_heads, w.head_dim, w.max_pages * w.page_size, 0)
+    for rep in range(2):
+        ds.append()
+        lse = torch.full((len(dec), w.num_q_heads), float("nan"), device="cuda")
+        out = pkv.pkv_paged_attn_decode_flags(ds.q_dec, ds.k_pool, ds.v_pool, ds.pt_dec, ds.len_dec, w.scale,
+                                              0, workspace=ws, out_lse=lse, flags=pkv.DECODE_METADATA_READY)
+        assert_close(bf16_to_f64(out)[sel], ref[sel], f"{name} metadata-ready decode, call {rep}")
+        assert_close(lse.cpu().numpy().astype(np.float64)[sel], ref_lse[sel], f"{name} lse, call {rep}")
+    check_no_flags(pkv)
+
+
 # ------------------------------------------------------- split-K combine API
 @pytest.mark.parametrize("d", [64, 128])
 def test_split_k_combine(pkv, d):
