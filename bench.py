@@ -197,6 +197,9 @@ class GpuWorkload:
         if dec:
             self.ws = pkv.decode_workspace(len(dec), w.num_q_heads, w.head_dim,
                                            w.max_pages * w.page_size, 0)
+        if pre and w.notes.get("attention") == "verify":
+            self.vws = pkv.verify_workspace(int(w.new_lens[pre].sum()), w.num_q_heads, w.head_dim,
+                                            w.max_pages * w.page_size, 0)
         # outputs: one packed device buffer per set, read back with one copy
         ospecs = {}
         if dec:
@@ -224,16 +227,25 @@ class GpuWorkload:
         return 1 + (1 if self.dec else 0) + (1 if self.pre else 0)
 
     def prefill_call(self, d=None, out=None):
+        """The chunk rows' attention: chunked prefill, or for the verify
+        workload the split-K short-chunk call."""
         d = self.dev if d is None else d
-        self.pkv.pkv_paged_attn_chunked_prefill(d["q_pre"], d["cu_q"], d["ctx_pre"], self.k_pool,
-                                                self.v_pool, d["pt_pre"], self.w.scale, self.max_q,
-                                                out=self.out_pre if out is None else out)
+        out = self.out_pre if out is None else out
+        if self.w.notes.get("attention") == "verify":
+            self.pkv.pkv_paged_attn_verify(d["q_pre"], d["cu_q"], d["ctx_pre"], self.k_pool, self.v_pool,
+                                           d["pt_pre"], self.w.scale, self.max_q, 0, workspace=self.vws, out=out)
+        else:
+            self.pkv.pkv_paged_attn_chunked_prefill(d["q_pre"], d["cu_q"], d["ctx_pre"], self.k_pool,
+                                                    self.v_pool, d["pt_pre"], self.w.scale, self.max_q, out=out)
 
     def decode_call(self, d=None, out=None):
         d = self.dev if d is None else d
-        self.pkv.pkv_paged_attn_decode(d["q_dec"], self.k_pool, self.v_pool, d["pt_dec"], d["len_dec"],
-                                       self.w.scale, 0, workspace=self.ws,
-                                       out=self.out_dec if out is None else out)
+        # the kernel just ahead (the append, the prefill or, in the timing
+        # loops, another decode) writes neither lengths nor page tables
+        self.pkv.pkv_paged_attn_decode_flags(d["q_dec"], self.k_pool, self.v_pool, d["pt_dec"], d["len_dec"],
+                                             self.w.scale, 0, workspace=self.ws,
+                                             out=self.out_dec if out is None else out,
+                                             flags=self.pkv.DECODE_METADATA_READY)
 
     def step(self, d, outs=None):
         """One pass of the hot path on device buffers d: kv_append of the
@@ -651,7 +663,7 @@ def main():
     head = measure(pkv, torch, HEADLINE, args.steps, args.warmup, dist, local)
     extra = {}
     names = [] if args.workloads == "none" else (
-        [n for n in ("tiny_decode", "mixed_prefill_decode", "splitk_long", "frag_large")]
+        [n for n in ("tiny_decode", "mixed_prefill_decode", "splitk_long", "frag_large", "spec_verify")]
         if args.workloads == "all" else [n for n in args.workloads.split(",") if n])
     for n in names:
         r = measure(pkv, torch, n, args.steps, args.warmup, dist, local)
@@ -663,14 +675,19 @@ def main():
             e.update({"decode_kv_bytes": r["kv_bytes_dec"], "decode_ms": r["dec_ms"],
                       "decode_kv_gbs": gbs, "decode_pct_of_8TBs": 100 * gbs / HBM_NOMINAL_GBS,
                       "decode_frac_of_measured_hbm": gbs / hbm})
-        if r["pre_ms"]:
+        if r["pre_ms"] and r["w"].notes.get("attention") == "verify":
+            gbs = r["kv_bytes_pre"] / (r["pre_ms"] / 1e3) / 1e9
+            e.update({"verify_kv_bytes": r["kv_bytes_pre"], "verify_ms": r["pre_ms"], "verify_kv_gbs": gbs,
+                      "verify_pct_of_8TBs": 100 * gbs / HBM_NOMINAL_GBS, "verify_frac_of_measured_hbm": gbs / hbm,
+                      "verify_tokens_per_s": world * r["tokens"] / (r["pre_ms"] / 1e3)})
+        elif r["pre_ms"]:
             tfs = r["flops_pre"] / (r["pre_ms"] / 1e3) / 1e12
             e.update({"prefill_ms": r["pre_ms"], "prefill_flops": r["flops_pre"],
                       "prefill_tflops": tfs, "prefill_frac_of_measured_bf16": tfs / tf_sust})
         e["step_kv_gbs"] = (r["kv_bytes_dec"] + r["kv_bytes_pre"]) / (r["ms_per_step"] / 1e3) / 1e9
         e["clocks"] = r["clocks"]
         extra[n] = e
-        if r["pre_ms"]:
+        if r["pre_ms"] and r["w"].notes.get("attention") != "verify":
             pre_roof = {"bound": "tensor", "achieved": r["flops_pre"] / (r["pre_ms"] / 1e3) / 1e12,
                         "peak": tf_sust, "unit": "TFLOP/s",
                         "traffic": profiled_traffic("prefill_mixed_prefill_decode"),
@@ -693,7 +710,8 @@ def main():
     cpu = None
     if world == 1 and args.cpu_budget > 0:
         # the oracle on the host cores, whole workloads, 1 thread and all cores
-        cpu = {n: oracle_times(n, "decode") for n in [HEADLINE] + [n for n in names if n != "mixed_prefill_decode"]}
+        cpu = {n: oracle_times(n, "prefill" if n == "spec_verify" else "decode")
+               for n in [HEADLINE] + [n for n in names if n != "mixed_prefill_decode"]}
         if "mixed_prefill_decode" in names:
             cpu["mixed_prefill_decode"] = {"decode": oracle_times("mixed_prefill_decode", "decode"),
                                            "prefill": oracle_times("mixed_prefill_decode", "prefill")}

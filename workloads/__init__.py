@@ -18,6 +18,10 @@ Shapes follow the workloads the pages describe:
                               lengths U[256,4096] in one batch.
   * "splitk_long"          - Llama-3.2-1B shapes (32/8 heads, d=64), 4 long
                               contexts 32k..128k, the flash-decoding case.
+  * "spec_verify"          - speculative-decoding verify: 64 requests of
+                              the Qwen3-4B layer, 4 query rows each (3 draft
+                              tokens + the last accepted one) at the end of
+                              contexts U[128,4096].
   * "frag_large"           - 256 requests, lognormal lengths (median 1536,
                               sigma 0.8, clipped [16,16384]), page 32, page
                               tables produced by an alloc/free trace over a
@@ -355,4 +359,17 @@ def make_workload(name: str, seed: int = 0, **over) -> Workload:
         return Workload(name, seed, Hq, Hkv, D, P, num_pages, table,
                         kv - 1, np.ones_like(kv), np.zeros(len(kv), bool),
                         notes={"trace": "grow-all / free 30% / regrow, LIFO free list"})
+    if name == "spec_verify":
+        # every request verifies q_len tokens (draft tokens plus the last
+        # accepted one) over its context: chunk rows at kv_len - q_len ..
+        # kv_len - 1
+        Hq, Hkv, D, P = over.get("num_q_heads", 32), over.get("num_kv_heads", 8), over.get("head_dim", 128), over.get("page_size", 16)
+        B, q_len = over.get("B", 64), over.get("q_len", 4)
+        kv = rng.integers(over.get("len_lo", 128), over.get("len_hi", 4096), size=B, endpoint=True).astype(np.int32)
+        need = int(sum((int(L) + P - 1) // P for L in kv))
+        num_pages = int(math.ceil(1.25 * need))
+        table = _permuted_tables(rng, kv, P, num_pages)
+        new = np.full(B, q_len, np.int32)
+        return Workload(name, seed, Hq, Hkv, D, P, num_pages, table, kv - new, new, np.ones(B, bool),
+                        k_rms_norm=True, notes={"attention": "verify"})
     raise ValueError(f"unknown workload {name!r}; known: {CONFIG_NAMES}")
