@@ -227,16 +227,17 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       const CUtensorMap* map = which ? &vmap : &kmap;
       const uint32_t dst = which ? sV(b) : sK(b);
       if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(pg.x * p.P * D * 2));
-      for (int pi = 0; pi < pg.x; ++pi) {
-        const int page = __shfl_sync(0xffffffffu, pg.y, pi);
-        if (lane == 0) {
-          if (which == 0 && static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages))
-            raise_flag(PKV_FLAG_BAD_PAGE);  // TMA reads zeros out of bounds
-          const int row = page * p.Hkv + g;
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(dst + h * LY::kKVHalf + pi * p.P * 128, map, 64 * h, 0, row, full);
-        }
+      __syncwarp();
+      // one box per lane, lane -> (page pi, 64-column half h): a TMA issue
+      // occupies its thread for ~130 cycles, so boxes issued by one lane go
+      // out one after another while boxes of different lanes go out together
+      constexpr int H = D / 64;
+      const int pi = lane / H, h = lane % H;
+      const int page = __shfl_sync(0xffffffffu, pg.y, pi & 31);
+      if (pi < pg.x) {
+        if (which == 0 && h == 0 && static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages))
+          raise_flag(PKV_FLAG_BAD_PAGE);  // TMA reads zeros out of bounds
+        tma_load_3d(dst + h * LY::kKVHalf + pi * p.P * 128, map, 64 * h, 0, page * p.Hkv + g, full);
       }
     };
     bool ok = true;
@@ -332,6 +333,11 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     const int pos_local = row / G, hh = row % G;
     const int qpos = pos_lo + pos_local;   // absolute position
     const bool row_valid = pos_local < rows_valid;
+    // a warp whose 32 rows all lie past the chunk (short chunks, the last
+    // tile of a chunk) computes no softmax: it waits for S (so it never runs
+    // ahead into the next phase), zeroes its share of a ragged V tile and
+    // counts itself done with P; its rows' P and O are never read out
+    const bool warp_idle = quad * 32 >= rows_valid * G;
     const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
@@ -339,6 +345,8 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
       if (!mbar_wait(bar(kSFull + b), (j >> 1) & 1)) { ok = false; break; }
+      const int key0 = (j0 + j) * kN;
+      if (!warp_idle) {
       tc_fence_after_sync();
       // raw scores of this row; hidden keys -> -inf (scale > 0, so the max
       // of raw scores gives the max of scaled ones)
@@ -353,7 +361,6 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(v[cc][e]);
       }
-      const int key0 = (j0 + j) * kN;
       if (key0 + kN - 1 > pos_lo || key0 + kN > kv_end) {  // diagonal or ragged tile
 #pragma unroll
         for (int e = 0; e < kN; ++e) {
@@ -411,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
         tmem_st_32x32b_x32(trow + (b ? kColS1 : kColS0) + cc * 32, w);
       }
       tmem_wait_st();
+      }  // !warp_idle
       if (key0 + kN > kv_end) {
         // ragged last tile: V rows past kv_end were not loaded (or hold
         // unused slots); zero them so 0 * garbage cannot reach O
@@ -427,12 +435,12 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       tc_fence_before_sync();
       mbar_arrive(bar(kPFull + b));
     }
-    const bool have_o = ok && nt >= 1 && mbar_wait(bar(kPVDone + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1);
+    const bool have_o = ok && !warp_idle && nt >= 1 && mbar_wait(bar(kPVDone + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1);
     const size_t qrow = static_cast<size_t>(q0 + qt * QPOS + pos_local);  // this thread's chunk row
     if (split_mode && split == 0 && g == 0 && hh == 0 && row_valid) p.num_splits[qrow] = req_splits;
     if (have_o) tc_fence_after_sync();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    if (to_partial && (have_o || (ok && nt == 0))) {
+    if (to_partial && !warp_idle && (have_o || (ok && nt == 0))) {
       // a partial normalised within this split (zero, lse -inf, when the
       // split holds none of the tile's keys), for the combine kernel
       const size_t prow = (qrow * p.Hq + g * G + hh) * p.splits + split;
