@@ -314,6 +314,49 @@ PKV_API int pkv_paged_attn_decode_static(const void* q, int32_t batch, int32_t n
                                          pkv_stream_t stream);
 
 /*
+ * pkv_mixed_workspace_bytes -- bytes of workspace pkv_paged_attn_mixed needs
+ * for batch_dec decode requests of at most max_kv_len keys (the decode
+ * workspace of the automatic split).
+ */
+PKV_API size_t pkv_mixed_workspace_bytes(int32_t batch_dec, int32_t num_q_heads, int32_t head_dim,
+                                         int32_t max_kv_len);
+
+/*
+ * pkv_paged_attn_mixed -- a continuous batch that mixes prefill chunks and
+ * decode requests in ONE persistent launch (tiny-llm source reading,
+ * "Continuous Batching": prefill and decode requests handled in the same
+ * round; "Chunked Prefill").  The CTAs, two per SM, pull work units from one
+ * queue: the chunks' query tiles first, heaviest request first, then the
+ * decode work cut into equal slices (the automatic split), so CTAs that
+ * finish their chunk tiles early stream decode KV while the last tiles run.
+ * No CTA waits for another.  Results are those of
+ * pkv_paged_attn_chunked_prefill (chunk rows) and pkv_paged_attn_decode with
+ * partition_tokens = 0 (decode rows).
+ *
+ *   chunk part   q_pre, cu_q_lens, batch_pre, total_q, max_q_len,
+ *                ctx_offsets, page_table_pre [batch_pre][max_pages_pre], out_pre:
+ *                as pkv_paged_attn_chunked_prefill
+ *   decode part  q_dec, batch_dec, page_table_dec [batch_dec][max_pages_dec],
+ *                kv_lens, out_dec, out_lse_dec (nullable): as
+ *                pkv_paged_attn_decode
+ *   workspace    pkv_mixed_workspace_bytes(...) bytes, ZERO-FILLED before
+ *                its first use, as the decode workspace (the call leaves its
+ *                counters at zero); calls sharing it must not overlap
+ *
+ * Either part may be empty.  Group size 8, or a batch whose decode plan
+ * does not fit two CTAs per SM, runs as the chunk kernel followed by the
+ * decode kernel (same results, two launches).
+ */
+PKV_API int pkv_paged_attn_mixed(const void* q_pre, const int32_t* cu_q_lens, int32_t batch_pre,
+                                 int32_t total_q, int32_t max_q_len, const int32_t* ctx_offsets,
+                                 const int32_t* page_table_pre, int32_t max_pages_pre,
+                                 const void* q_dec, int32_t batch_dec, const int32_t* page_table_dec,
+                                 int32_t max_pages_dec, const int32_t* kv_lens, int32_t num_q_heads,
+                                 const void* k_pool, const void* v_pool, pkv_pool_desc pool,
+                                 float scale, void* workspace, size_t workspace_bytes, void* out_pre,
+                                 void* out_dec, float* out_lse_dec, pkv_stream_t stream);
+
+/*
  * pkv_qk_norm_rope_append -- the step before attention in one kernel: the
  * separate RMSNorm of each projected query and key head row, rotary position
  * encoding of both, and the write of the new K row (and the V row, as it is)

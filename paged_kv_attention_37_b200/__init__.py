@@ -29,7 +29,7 @@ __all__ = [
     "pkv_status_string", "pkv_device_error_flags", "decode_workspace",
     "pkv_paged_attn_decode_static", "pkv_qk_norm_rope_append", "pkv_kv_append_cow",
     "pkv_verify_workspace_bytes", "verify_workspace", "pkv_paged_attn_verify", "pkv_paged_attn_decode_flags",
-    "DECODE_METADATA_READY",
+    "DECODE_METADATA_READY", "pkv_mixed_workspace_bytes", "mixed_workspace", "pkv_paged_attn_mixed",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -85,6 +85,11 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_attn_decode_flags.argtypes = [P, I32, I32, P, P, _PoolDesc, P, I32, P, F32, I32, P, SZ,
                                                 P, P, ctypes.c_uint32, P]
     lib.pkv_paged_attn_decode_flags.restype = ctypes.c_int
+    lib.pkv_mixed_workspace_bytes.argtypes = [I32, I32, I32, I32]
+    lib.pkv_mixed_workspace_bytes.restype = SZ
+    lib.pkv_paged_attn_mixed.argtypes = [P, P, I32, I32, I32, P, P, I32, P, I32, P, I32, P, I32, P, P, _PoolDesc,
+                                         F32, P, SZ, P, P, P, P]
+    lib.pkv_paged_attn_mixed.restype = ctypes.c_int
     lib.pkv_verify_workspace_bytes.argtypes = [I32, I32, I32, I32, I32]
     lib.pkv_verify_workspace_bytes.restype = SZ
     lib.pkv_paged_attn_verify.argtypes = [P, P, I32, I32, I32, I32, P, P, P, _PoolDesc, P, I32, F32, I32, P,
@@ -248,6 +253,54 @@ def pkv_paged_attn_chunked_prefill(q, cu_q_lens, ctx_offsets, k_pool, v_pool, pa
         _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table), page_table.shape[1],
         float(scale), _ptr(out), _stream(stream)))
     return out
+
+
+def pkv_mixed_workspace_bytes(batch_dec, num_q_heads, head_dim, max_kv_len) -> int:
+    return int(_lib.pkv_mixed_workspace_bytes(batch_dec, num_q_heads, head_dim, max_kv_len))
+
+
+def mixed_workspace(batch_dec, num_q_heads, head_dim, max_kv_len, device=None):
+    """A zero-filled workspace of the size pkv_paged_attn_mixed needs."""
+    n = pkv_mixed_workspace_bytes(batch_dec, num_q_heads, head_dim, max_kv_len)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def pkv_paged_attn_mixed(q_pre, cu_q_lens, ctx_offsets, page_table_pre, max_q_len, q_dec, page_table_dec,
+                         kv_lens, k_pool, v_pool, scale, workspace=None, out_pre=None, out_dec=None,
+                         out_lse_dec=None, stream=None):
+    """Prefill chunks (q_pre [total_q, Hq, d], cu_q_lens, ctx_offsets) and decode
+    requests (q_dec [B, Hq, d], kv_lens) of one batch in a single persistent
+    launch; returns (out_pre, out_dec)."""
+    _need(q_pre, "q_pre", torch.bfloat16, 3)
+    _need(cu_q_lens, "cu_q_lens", torch.int32, 1)
+    _need(ctx_offsets, "ctx_offsets", torch.int32, 1)
+    _need(page_table_pre, "page_table_pre", torch.int32, 2)
+    _need(q_dec, "q_dec", torch.bfloat16, 3)
+    _need(page_table_dec, "page_table_dec", torch.int32, 2)
+    _need(kv_lens, "kv_lens", torch.int32, 1)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    total_q, hq, d = q_pre.shape
+    bp, bd = ctx_offsets.shape[0], q_dec.shape[0]
+    if cu_q_lens.shape[0] != bp + 1 or page_table_pre.shape[0] != bp:
+        raise ValueError("cu_q_lens must have B+1 entries and page_table_pre B rows")
+    if page_table_dec.shape[0] != bd or kv_lens.shape[0] != bd or q_dec.shape[1:] != q_pre.shape[1:]:
+        raise ValueError("decode tensors disagree on the batch or the head shape")
+    if workspace is None:
+        workspace = mixed_workspace(bd, hq, d, page_table_dec.shape[1] * k_pool.shape[2], q_pre.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    out_pre = torch.empty_like(q_pre) if out_pre is None else out_pre
+    out_dec = torch.empty_like(q_dec) if out_dec is None else out_dec
+    _need(out_pre, "out_pre", torch.bfloat16, 3)
+    _need(out_dec, "out_dec", torch.bfloat16, 3)
+    if out_lse_dec is not None:
+        _need(out_lse_dec, "out_lse_dec", torch.float32, 2)
+    _check("pkv_paged_attn_mixed", _lib.pkv_paged_attn_mixed(
+        _ptr(q_pre), _ptr(cu_q_lens), bp, total_q, int(max_q_len), _ptr(ctx_offsets), _ptr(page_table_pre),
+        page_table_pre.shape[1], _ptr(q_dec), bd, _ptr(page_table_dec), page_table_dec.shape[1],
+        _ptr(kv_lens), hq, _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), float(scale), _ptr(workspace),
+        workspace.numel(), _ptr(out_pre), _ptr(out_dec), _ptr(out_lse_dec), _stream(stream)))
+    return out_pre, out_dec
 
 
 def pkv_verify_workspace_bytes(total_q, num_q_heads, head_dim, max_kv_len, partition_tokens=0) -> int:

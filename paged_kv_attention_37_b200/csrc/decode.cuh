@@ -381,19 +381,24 @@ __device__ __forceinline__ void merge_regs(const Params& p, int r, int g, int ns
   }
 }
 
-template <int D, int G, int NS, int MAXW>
-__global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p) {
+// The body of the decode kernel, for CTA number `cta` of `ncta` CTAs that
+// share the batch, with W decode warps; warps of the CTA past W (when the
+// CTA has more, as in the mixed kernel) only take part in its barrier.
+// `smem` is the CTA's dynamic shared memory.  kLean: 8 elements of d per
+// lane in the score phase even where 16 would fit, which frees the
+// registers of half the query rows (for kernels that hold other work).
+template <int D, int G, int NS, bool kLean = false>
+__device__ __forceinline__ void decode_body(const Params& p, int cta, int ncta, int W, uint8_t* smem) {
   using LY = Layout<D, G, NS>;
   constexpr int kFI = kMergeFanIn<D>;  // merge-tree fan-in
   using CK = Chunk<D>;
   constexpr int kTok = CK::kTokens;
   // score phase: E elements of d per lane (16 at d=128 unless G=8, whose
   // doubled query registers would not fit; else 8), T lanes per token
-  constexpr int E = (D == 128 && G <= 4) ? 16 : 8;
+  constexpr int E = (D == 128 && G <= 4 && !kLean) ? 16 : 8;
   constexpr int T = D / E, TPS = 32 / T, STEPS = kTok / TPS;
   constexpr int LG = ilog2(G), LT = ilog2(T);
   constexpr int DPL = D / 32;  // P.V output elements per lane
-  const int W = blockDim.x >> 5;
   const int log2P = 31 - __clz(p.P);  // P is a power of two
   static_assert((T == 8 || T == 16) && (D == 64 || D == 128), "head_dim 64 or 128");
   static_assert(NS >= 2, "at least two stages per warp");
@@ -406,7 +411,6 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   const bool early = p.meta_ready != 0 && p.partition == 0;
   if (!early) pdl_wait();
 
-  extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t* misc = reinterpret_cast<int32_t*>(smem + W * LY::kWarpBytes);
   int32_t* lens = misc + 4;
@@ -419,11 +423,11 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   ChunkInfo* fifo = reinterpret_cast<ChunkInfo*>(wb + LY::kFifoOff);
   ItemInfo* items = reinterpret_cast<ItemInfo*>(wb + LY::kItemOff);
   ItemInfo* climb = reinterpret_cast<ItemInfo*>(wb + LY::kClimbOff);
-  if (lane < kClimbSlots) climb[lane].r = -1;
+  if (warp < W && lane < kClimbSlots) climb[lane].r = -1;
   float* pb = reinterpret_cast<float*>(wb + LY::kPbOff);
 
   if constexpr (!kCpAsync) {
-    if (lane == 0) {
+    if (warp < W && lane == 0) {
       for (int i = 0; i < NS; ++i) mbar_init(full_bar(i), 1);
       fence_barrier_init();
     }
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       }
       lens[r] = L;
     }
-    if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) raise_flag(PKV_FLAG_BAD_LENGTH);
+    if (__any_sync(0xffffffffu, bad) && lane == 0 && cta == 0) raise_flag(PKV_FLAG_BAD_LENGTH);
     int part = 0;
     if (p.partition > 0) {
       part = p.partition;
@@ -473,7 +477,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
       }
       // slices of floor(Q/Weff) or one quantum more, at least kMinShare tokens
       const int weff = static_cast<int>(
-          min(static_cast<long long>(gridDim.x) * W, max(1ll, static_cast<long long>(runF) / (kMinShare / kPartitionQuantum))));
+          min(static_cast<long long>(ncta) * W, max(1ll, static_cast<long long>(runF) / (kMinShare / kPartitionQuantum))));
       if (lane == 0) {
         prefF[0] = 0;
         misc[0] = weff;  // warps with a slice
@@ -488,7 +492,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
         const int L = lens[r];
         nf = (L / part) * p.Hkv;
         nr = (L % part != 0 || L == 0) ? p.Hkv : 0;
-        if (blockIdx.x == 0) p.num_splits[r] = L == 0 ? 1 : (L + part - 1) / part;
+        if (cta == 0) p.num_splits[r] = L == 0 ? 1 : (L + part - 1) / part;
       }
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -518,6 +522,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   // let a dependent launch (the combine kernel) be scheduled now; it waits
   // for this whole grid to finish before reading anything
   pdl_launch_dependents();
+  if (warp >= W) return;
   // misc[0] holds one value with two readings: under a fixed partition its
   // length in tokens (part), under the automatic split the number of warps
   // that get a slice (weff)
@@ -526,7 +531,7 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   // automatic split: warp w < Weff takes quanta [floor(w*Q/Weff),
   // floor((w+1)*Q/Weff)) of the Q = nF quanta; the slice holding quantum x
   // is floor(((x+1)*Weff - 1) / Q)
-  const int wid = blockIdx.x * W + warp;
+  const int wid = cta * W + warp;
   auto slice_start = [&](int w) { return static_cast<int>(static_cast<long long>(w) * nF / weff); };
   auto slice_of = [&](int x) { return static_cast<int>((static_cast<long long>(x + 1) * weff - 1) / nF); };
   int bq = balanced && wid < weff ? slice_start(wid) : 0;
@@ -982,12 +987,18 @@ __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p)
   }
   if (lane == 0) {
     __threadfence();
-    if (atomicAdd(&p.counters[1], 1u) == gridDim.x * W - 1) {
+    if (atomicAdd(&p.counters[1], 1u) == static_cast<uint32_t>(ncta * W - 1)) {
       p.counters[0] = 0;
       p.counters[1] = 0;
       __threadfence();
     }
   }
+}
+
+template <int D, int G, int NS, int MAXW>
+__global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  decode_body<D, G, NS>(p, blockIdx.x, gridDim.x, blockDim.x >> 5, smem);
 }
 
 // Merge split partials.  One CTA per (request, query head) row; its warps

@@ -13,6 +13,7 @@
 #include "cow.cuh"
 #include "decode.cuh"
 #include "kv_append.cuh"
+#include "mixed.cuh"
 #include "prefill.cuh"
 #include "prologue.cuh"
 
@@ -341,47 +342,36 @@ VerifyLayout verify_layout(int32_t total_q, int32_t Hq, int32_t D, int32_t max_k
   return v;
 }
 
-// Chunked prefill (split_tokens = 0) or its split-K form (split_tokens =
-// the partition, -1 = automatic; workspace as verify_layout).
-int run_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t num_q_heads, int32_t total_q,
-                int32_t max_q_len, const int32_t* ctx_offsets, const void* k_pool, const void* v_pool,
-                const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages, float scale,
-                int32_t split_tokens, void* workspace, size_t workspace_bytes, void* out, cudaStream_t s) {
+// A checked chunk launch: the kernel's parameters, the three tensor maps and
+// the GQA group.
+struct PrefillLaunch {
+  pkv::prefill::Params prm;
+  CUtensorMap qmap, kmap, vmap;
+  int group = 0;
+};
+
+// Host-side checks of a chunk call and its parameters (no split).  Returns
+// PKV_OK, kNothingToDo for an empty call (after the shape checks), or an
+// error status.
+constexpr int kNothingToDo = 1;
+
+int build_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t num_q_heads, int32_t total_q,
+                  int32_t max_q_len, const int32_t* ctx_offsets, const void* k_pool, const void* v_pool,
+                  const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages, float scale, void* out,
+                  PrefillLaunch* pl) {
   if (batch < 0 || total_q < 0 || max_q_len < 0 || max_pages <= 0) return PKV_ERR_BAD_SHAPE;
   int st = check_pool(pool);
   if (st != PKV_OK) return st;
-  int group = 0;
-  if ((st = check_heads(num_q_heads, pool, &group)) != PKV_OK) return st;
+  if ((st = check_heads(num_q_heads, pool, &pl->group)) != PKV_OK) return st;
   if (!std::isfinite(scale) || !(scale > 0.f)) return PKV_ERR_BAD_SHAPE;
   if (static_cast<long long>(max_pages) * pool.page_size > (1ll << 30)) return PKV_ERR_BAD_SHAPE;
-  if (batch == 0 || total_q == 0 || max_q_len == 0) return PKV_OK;
+  if (batch == 0 || total_q == 0 || max_q_len == 0) return kNothingToDo;
   if (!q || !cu_q_lens || !ctx_offsets || !k_pool || !v_pool || !page_table || !out)
     return PKV_ERR_NULL_POINTER;
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
     return PKV_ERR_MISALIGNED;
-  VerifyLayout vl;
-  if (split_tokens != 0) {
-    vl = verify_layout(total_q, num_q_heads, pool.head_dim, max_pages * pool.page_size,
-                       split_tokens < 0 ? 0 : split_tokens);
-    if (workspace == nullptr || workspace_bytes < vl.total) return PKV_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
-  }
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != PKV_OK) return st;
-  const int D = pool.head_dim;
-  const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
-  const int qpos = pkv::prefill::kRowsPerCta / group;
-  CUtensorMap qmap, kmap, vmap;
-  if ((st = make_map(&qmap, q, D, num_q_heads, total_q, D * 2ull, static_cast<uint64_t>(num_q_heads) * D * 2, 64,
-                     group, qpos, true)) != PKV_OK)
-    return st;
-  if ((st = make_map(&kmap, k_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
-                     pool.page_size, 1, true)) != PKV_OK)
-    return st;
-  if ((st = make_map(&vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
-                     pool.page_size, 1, true)) != PKV_OK)
-    return st;
-  pkv::prefill::Params prm;
+  const int qpos = pkv::prefill::kRowsPerCta / pl->group;
+  pkv::prefill::Params& prm = pl->prm;
   prm.cu_q_lens = cu_q_lens;
   prm.ctx_offsets = ctx_offsets;
   prm.page_table = page_table;
@@ -393,12 +383,57 @@ int run_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t 
   prm.max_pages = max_pages;
   prm.num_pages = pool.num_pages;
   prm.total_q = total_q;
+  prm.qtiles = static_cast<int32_t>((static_cast<long long>(max_q_len) + qpos - 1) / qpos);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.partition = 0;
   prm.splits = 1;
   prm.part_o = nullptr;
   prm.part_lse = nullptr;
   prm.num_splits = nullptr;
+  return PKV_OK;
+}
+
+// The TMA maps of a checked chunk launch (after every argument check: the
+// driver's encoder is the first call that can fail for reasons of its own).
+int make_prefill_maps(const void* q, const void* k_pool, const void* v_pool, const pkv_pool_desc& pool,
+                      int32_t num_q_heads, int32_t total_q, PrefillLaunch* pl) {
+  const int D = pool.head_dim;
+  const uint64_t rows = static_cast<uint64_t>(pool.num_pages) * pool.num_kv_heads;
+  const int qpos = pkv::prefill::kRowsPerCta / pl->group;
+  int st;
+  if ((st = make_map(&pl->qmap, q, D, num_q_heads, total_q, D * 2ull, static_cast<uint64_t>(num_q_heads) * D * 2,
+                     64, pl->group, qpos, true)) != PKV_OK)
+    return st;
+  if ((st = make_map(&pl->kmap, k_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
+                     pool.page_size, 1, true)) != PKV_OK)
+    return st;
+  return make_map(&pl->vmap, v_pool, D, pool.page_size, rows, D * 2ull, pool.page_size * D * 2ull, 64,
+                  pool.page_size, 1, true);
+}
+
+// Chunked prefill (split_tokens = 0) or its split-K form (split_tokens =
+// the partition, -1 = automatic; workspace as verify_layout).
+int run_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t num_q_heads, int32_t total_q,
+                int32_t max_q_len, const int32_t* ctx_offsets, const void* k_pool, const void* v_pool,
+                const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages, float scale,
+                int32_t split_tokens, void* workspace, size_t workspace_bytes, void* out, cudaStream_t s) {
+  PrefillLaunch pl;
+  int st = build_prefill(q, cu_q_lens, batch, num_q_heads, total_q, max_q_len, ctx_offsets, k_pool, v_pool, pool,
+                         page_table, max_pages, scale, out, &pl);
+  if (st == kNothingToDo) return PKV_OK;
+  if (st != PKV_OK) return st;
+  VerifyLayout vl;
+  if (split_tokens != 0) {
+    vl = verify_layout(total_q, num_q_heads, pool.head_dim, max_pages * pool.page_size,
+                       split_tokens < 0 ? 0 : split_tokens);
+    if (workspace == nullptr || workspace_bytes < vl.total) return PKV_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  }
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  if ((st = make_prefill_maps(q, k_pool, v_pool, pool, num_q_heads, total_q, &pl)) != PKV_OK) return st;
+  const int D = pool.head_dim;
+  pkv::prefill::Params& prm = pl.prm;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (split_tokens != 0) {
     prm.partition = vl.partition;
@@ -410,8 +445,8 @@ int run_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t 
     // "one split" to the combine, which then leaves them alone
     if (cudaMemsetAsync(prm.num_splits, 0, static_cast<size_t>(total_q) * 4, s) != cudaSuccess) return PKV_ERR_CUDA;
   }
-  st = D == 128 ? dispatch_prefill_group<128>(group, prm, qmap, kmap, vmap, max_q_len, s)
-                : dispatch_prefill_group<64>(group, prm, qmap, kmap, vmap, max_q_len, s);
+  st = D == 128 ? dispatch_prefill_group<128>(pl.group, prm, pl.qmap, pl.kmap, pl.vmap, max_q_len, s)
+                : dispatch_prefill_group<64>(pl.group, prm, pl.qmap, pl.kmap, pl.vmap, max_q_len, s);
   if (st != PKV_OK || split_tokens == 0) return st;
   // merge the rows whose request was split (rows of single-split requests
   // were written by the kernel itself)
@@ -460,15 +495,12 @@ int check_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* 
   return PKV_OK;
 }
 
-// Launch a checked decode call on workspace ws (at least dp.wl.total bytes,
-// 256-byte aligned).
-int run_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool, const void* v_pool,
-               const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages,
-               const int32_t* kv_lens, float scale, int32_t partition_tokens, const DecodePlan& dp,
-               void* workspace, void* out, float* out_lse, uint32_t flags, cudaStream_t s) {
-  DeviceInfo dev;
-  int st;
-  if ((st = current_device(&dev)) != PKV_OK) return st;
+// The decode kernel's parameters for a checked call on workspace ws (at
+// least dp.wl.total bytes, 256-byte aligned).
+pkv::decode::Params fill_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool,
+                                const void* v_pool, const pkv_pool_desc& pool, const int32_t* page_table,
+                                int32_t max_pages, const int32_t* kv_lens, float scale, int32_t partition_tokens,
+                                const DecodePlan& dp, void* workspace, void* out, float* out_lse, uint32_t flags) {
   const WorkspaceLayout& wl = dp.wl;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   pkv::decode::Params prm;
@@ -495,9 +527,67 @@ int run_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_
   prm.merge_nodes = dp.ss.nodes;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.meta_ready = (flags & PKV_DECODE_METADATA_READY) ? 1 : 0;
-  if ((st = prepare_workspace(workspace, wl.zero_bytes, s)) != PKV_OK) return st;
+  return prm;
+}
+
+// Launch a checked decode call on workspace ws (at least dp.wl.total bytes,
+// 256-byte aligned).
+int run_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool, const void* v_pool,
+               const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages,
+               const int32_t* kv_lens, float scale, int32_t partition_tokens, const DecodePlan& dp,
+               void* workspace, void* out, float* out_lse, uint32_t flags, cudaStream_t s) {
+  DeviceInfo dev;
+  int st;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  const pkv::decode::Params prm = fill_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages,
+                                              kv_lens, scale, partition_tokens, dp, workspace, out, out_lse, flags);
+  if ((st = prepare_workspace(workspace, dp.wl.zero_bytes, s)) != PKV_OK) return st;
   if (pool.head_dim == 128) return dispatch_decode_group<128>(dp.group, prm, dev.sm_count, s);
   return dispatch_decode_group<64>(dp.group, prm, dev.sm_count, s);
+}
+
+// One persistent launch of a mixed batch (chunks and decode requests):
+// returns kNothingToDo when this group size or shared-memory footprint does
+// not allow two CTAs per SM, and the caller runs the two kernels instead.
+template <int D, int G>
+int launch_mixed(const PrefillLaunch& pl, const pkv::decode::Params& dprm, uint32_t* queue, int sm_count,
+                 cudaStream_t s) {
+  if constexpr (G > 4) {
+    return kNothingToDo;  // the decode body at G = 8 needs more registers than two CTAs per SM leave
+  } else {
+    using DL = pkv::decode::Layout<D, G, 2>;
+    const size_t smem = std::max<size_t>(pkv::prefill::smem_bytes<D>(), DL::bytes(pkv::mixed::kDecodeWarps, dprm.B));
+    auto kernel = pkv::mixed::mixed_kernel<D, G>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+      return PKV_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, pkv::prefill::kThreads, smem) != cudaSuccess)
+      return PKV_ERR_CUDA;
+    if (per_sm < 2) return kNothingToDo;
+    pkv::mixed::Params mp;
+    mp.pre = pl.prm;
+    mp.dec = dprm;
+    const long long units = static_cast<long long>(pl.prm.qtiles) * pl.prm.Hkv * pl.prm.B;
+    if (units > 0x3FFFFFFFll) return PKV_ERR_BAD_SHAPE;
+    mp.pre_units = static_cast<int32_t>(units);
+    mp.dec_units = 2 * sm_count;
+    mp.queue = queue;
+    return launch_pdl(kernel, dim3(2 * sm_count), dim3(pkv::prefill::kThreads), smem, s, pl.qmap, pl.kmap, pl.vmap,
+                      mp);
+  }
+}
+
+template <int D>
+int dispatch_mixed_group(const PrefillLaunch& pl, const pkv::decode::Params& dprm, uint32_t* queue, int sm_count,
+                         cudaStream_t s) {
+  switch (pl.group) {
+    case 1: return launch_mixed<D, 1>(pl, dprm, queue, sm_count, s);
+    case 2: return launch_mixed<D, 2>(pl, dprm, queue, sm_count, s);
+    case 4: return launch_mixed<D, 4>(pl, dprm, queue, sm_count, s);
+    case 8: return launch_mixed<D, 8>(pl, dprm, queue, sm_count, s);
+  }
+  return PKV_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -624,6 +714,60 @@ int pkv_paged_attn_verify(const void* q, const int32_t* cu_q_lens, int32_t batch
   return run_prefill(q, cu_q_lens, batch, num_q_heads, total_q, max_q_len, ctx_offsets, k_pool, v_pool, pool,
                      page_table, max_pages, scale, partition_tokens == 0 ? -1 : partition_tokens, workspace,
                      workspace_bytes, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t pkv_mixed_workspace_bytes(int32_t batch_dec, int32_t num_q_heads, int32_t head_dim, int32_t max_kv_len) {
+  return pkv_decode_workspace_bytes(std::max<int32_t>(batch_dec, 1), num_q_heads, head_dim, max_kv_len, 0);
+}
+
+int pkv_paged_attn_mixed(const void* q_pre, const int32_t* cu_q_lens, int32_t batch_pre, int32_t total_q,
+                         int32_t max_q_len, const int32_t* ctx_offsets, const int32_t* page_table_pre,
+                         int32_t max_pages_pre, const void* q_dec, int32_t batch_dec,
+                         const int32_t* page_table_dec, int32_t max_pages_dec, const int32_t* kv_lens,
+                         int32_t num_q_heads, const void* k_pool, const void* v_pool, pkv_pool_desc pool,
+                         float scale, void* workspace, size_t workspace_bytes, void* out_pre, void* out_dec,
+                         float* out_lse_dec, pkv_stream_t stream) {
+  PrefillLaunch pl;
+  const int stp = build_prefill(q_pre, cu_q_lens, batch_pre, num_q_heads, total_q, max_q_len, ctx_offsets, k_pool,
+                                v_pool, pool, page_table_pre, max_pages_pre, scale, out_pre, &pl);
+  if (stp < 0) return stp;
+  DecodePlan dp;
+  int st = check_decode(q_dec, batch_dec, num_q_heads, k_pool, v_pool, pool, page_table_dec, max_pages_dec, kv_lens,
+                        scale, 0, out_dec, &dp);
+  if (st != PKV_OK) return st;
+  const bool has_pre = stp == PKV_OK, has_dec = batch_dec > 0;
+  if (has_dec) {
+    if (workspace == nullptr || workspace_bytes < dp.wl.total) return PKV_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  }
+  if (!has_pre && !has_dec) return PKV_OK;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  if (has_pre && (st = make_prefill_maps(q_pre, k_pool, v_pool, pool, num_q_heads, total_q, &pl)) != PKV_OK)
+    return st;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  const int D = pool.head_dim;
+  if (!has_dec)
+    return D == 128 ? dispatch_prefill_group<128>(pl.group, pl.prm, pl.qmap, pl.kmap, pl.vmap, max_q_len, s)
+                    : dispatch_prefill_group<64>(pl.group, pl.prm, pl.qmap, pl.kmap, pl.vmap, max_q_len, s);
+  const pkv::decode::Params dprm = fill_decode(q_dec, batch_dec, num_q_heads, k_pool, v_pool, pool, page_table_dec,
+                                               max_pages_dec, kv_lens, scale, 0, dp, workspace, out_dec,
+                                               out_lse_dec, 0u);
+  if ((st = prepare_workspace(workspace, dp.wl.zero_bytes, s)) != PKV_OK) return st;
+  if (has_pre) {
+    // the queue counters sit after the decode kernel's two in the workspace's
+    // counter block, which every completed call leaves zero
+    uint32_t* queue = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + dp.wl.counters) + 2;
+    st = D == 128 ? dispatch_mixed_group<128>(pl, dprm, queue, dev.sm_count, s)
+                  : dispatch_mixed_group<64>(pl, dprm, queue, dev.sm_count, s);
+    if (st != kNothingToDo) return st;
+    // this batch runs as two kernels
+    st = D == 128 ? dispatch_prefill_group<128>(pl.group, pl.prm, pl.qmap, pl.kmap, pl.vmap, max_q_len, s)
+                  : dispatch_prefill_group<64>(pl.group, pl.prm, pl.qmap, pl.kmap, pl.vmap, max_q_len, s);
+    if (st != PKV_OK) return st;
+  }
+  if (D == 128) return dispatch_decode_group<128>(dp.group, dprm, dev.sm_count, s);
+  return dispatch_decode_group<64>(dp.group, dprm, dev.sm_count, s);
 }
 
 int pkv_qk_norm_rope_append(const void* q, const void* k, const void* v, int32_t num_tokens,

@@ -57,9 +57,6 @@ struct Params {
   int32_t* num_splits;  // [total_q]: splits of each chunk row's request
 };
 
-#ifndef PKV_PREFILL_ORDER
-#define PKV_PREFILL_ORDER 1
-#endif
 
 template <int D, int BN>
 struct Layout {
@@ -84,10 +81,49 @@ constexpr size_t smem_bytes();
 enum Bar { kQ = 0, kKFull = 1, kKEmpty = 3, kVFull = 5, kVEmpty = 7, kSFull = 9, kPFull = 11,
            kPVDone = 13, kFinal = 15 };
 
-template <int D, int G, int BN>
-__global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, const Params p) {
+// Rows of a chunk and keys its last row sees: the CTAs' weight ranking key.
+__device__ __forceinline__ long long chunk_weight(const Params& p, int r) {
+  const int q0 = p.cu_q_lens[r], q1 = p.cu_q_lens[r + 1], c = p.ctx_offsets[r];
+  return (q1 >= q0 && c >= 0) ? static_cast<long long>(q1 - q0) * (c + q1 - q0) : 0;
+}
+
+// The request that comes rank-th when the requests are ordered by decreasing
+// work (rows x keys of the last row, ties by index).  CTAs take the chunks
+// heaviest request first, so the longest-running CTAs start early instead of
+// being left alone at the end.  The CTA's threads stage one weight each in
+// shared memory and each ranks its own request against the staged ones;
+// batches larger than the CTA keep their own order.  Every thread of the
+// CTA calls it.
+constexpr int kRankMax = 192;  // = the chunk kernel's threads
+__device__ __forceinline__ int request_by_weight(const Params& p, int rank) {
+  __shared__ long long wt[kRankMax];
+  __shared__ int chosen;
+  if (p.B > kRankMax || p.B > static_cast<int>(blockDim.x)) return rank;
+  const int c = threadIdx.x;
+  if (c < p.B) wt[c] = chunk_weight(p, c);
+  if (c == 0) chosen = rank;
+  __syncthreads();
+  if (c < p.B) {
+    const long long wc = wt[c];
+    int k = 0;
+    for (int o = 0; o < p.B; ++o) k += (wt[o] > wc) || (wt[o] == wc && o < c);
+    if (k == rank) chosen = c;
+  }
+  __syncthreads();
+  const int r = chosen;
+  __syncthreads();  // wt and chosen are reused by the next call
+  return r;
+}
+
+// The body of the chunk kernel for work unit `unit` (what a CTA of the
+// standalone launch does for blockIdx.x = unit), on the CTA's dynamic shared
+// memory `smem_raw`.  The caller has waited for the kernel ahead.  kOnce: the
+// CTA runs one unit and gives up its TMEM allocation permit after it
+// allocates; a persistent CTA (one allocation per unit) keeps it.
+template <int D, int G, int BN, bool kOnce = true>
+__device__ __forceinline__ void prefill_body(const CUtensorMap* qmap_p, const CUtensorMap* kmap_p,
+                                             const CUtensorMap* vmap_p, const Params& p, int unit,
+                                             uint8_t* smem_raw) {
   using LY = Layout<D, BN>;
   constexpr int kN = BN;        // keys per tile
   constexpr int kTmemCols = LY::kTmemCols;
@@ -95,29 +131,15 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
   constexpr int QPOS = kM / G;  // chunk positions per tile
   constexpr uint32_t kIdescS = idesc_bf16_f32(kM, kN, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, D, false, true);
-  // launched as a programmatic dependent (see pdl_wait): nothing global is
-  // read before the kernel ahead of it has completed
-  pdl_wait();
-  pdl_launch_dependents();
-
-  // ---- which tile.  Order 1: the query tiles of one (request, KV head) are
+  // ---- which tile: the query tiles of one (request, KV head) are
   // adjacent, heaviest (last) first, so the CTAs that read the same keys run
-  // together and share them through L2.  Order 0: heaviest tiles of every
-  // request first.
-  int r, g, qt_rev;
-  const int split = blockIdx.x % p.splits;  // the splits of a query tile are adjacent
-  const int bx = blockIdx.x / p.splits;
-  if (PKV_PREFILL_ORDER == 1) {
-    qt_rev = bx % p.qtiles;
-    const int rest = bx / p.qtiles;
-    g = rest % p.Hkv;
-    r = rest / p.Hkv;
-  } else {
-    r = bx % p.B;
-    const int rest = bx / p.B;
-    g = rest % p.Hkv;
-    qt_rev = rest / p.Hkv;
-  }
+  // together and share them through L2; requests by decreasing work; the
+  // splits of one query tile adjacent
+  const int split = unit % p.splits;
+  const int bx = unit / p.splits;
+  const int qt_rev = bx % p.qtiles;
+  const int g = (bx / p.qtiles) % p.Hkv;
+  const int r = request_by_weight(p, bx / p.qtiles / p.Hkv);
   const int q0 = p.cu_q_lens[r], q1 = p.cu_q_lens[r + 1];
   const int n_r = q1 - q0;
   if (q0 < 0 || n_r < 0 || q1 > p.total_q) {
@@ -151,7 +173,6 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 
   // 128-byte swizzle atoms need 1024-byte alignment; the declaration asks
   // for it, and a misaligned base (never expected) is refused, not used
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_addr(smem);
   if (sbase & 1023u) {
@@ -176,7 +197,12 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     mbar_init(bar(kFinal), 1);
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(smem_addr(smem + LY::kTmemSlotOff), kTmemCols);
+  if (warp == 1) {
+    if constexpr (kOnce)
+      tmem_alloc(smem_addr(smem + LY::kTmemSlotOff), kTmemCols);
+    else
+      tmem_alloc_again(smem_addr(smem + LY::kTmemSlotOff), kTmemCols);
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -190,13 +216,13 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     // ============================ TMA producer ============================
     const int32_t* ptab = p.page_table + static_cast<size_t>(r) * p.max_pages;
     if (lane == 0) {
-      prefetch_tensormap(&qmap);
-      prefetch_tensormap(&kmap);
-      prefetch_tensormap(&vmap);
+      prefetch_tensormap(qmap_p);
+      prefetch_tensormap(kmap_p);
+      prefetch_tensormap(vmap_p);
       mbar_arrive_expect_tx(bar(kQ), kM * D * 2);
 #pragma unroll
       for (int h = 0; h < D / 64; ++h)
-        tma_load_3d(sQ + h * LY::kQHalf, &qmap, 64 * h, g * G, q0 + qt * QPOS, bar(kQ));
+        tma_load_3d(sQ + h * LY::kQHalf, qmap_p, 64 * h, g * G, q0 + qt * QPOS, bar(kQ));
     }
     // K of tile j only waits for its stage (freed when S of tile j-2 is
     // done); V trails one tile behind, since P.V of a tile runs after its
@@ -224,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     auto issue_tile = [&](int j, int2 pg, int which) {  // which: 0 = K, 1 = V
       const int b = j & 1;
       const uint32_t full = bar((which ? kVFull : kKFull) + b);
-      const CUtensorMap* map = which ? &vmap : &kmap;
+      const CUtensorMap* map = which ? vmap_p : kmap_p;
       const uint32_t dst = which ? sV(b) : sK(b);
       if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(pg.x * p.P * D * 2));
       __syncwarp();
@@ -494,6 +520,18 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+template <int D, int G, int BN>
+__global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // launched as a programmatic dependent (see pdl_wait): nothing global is
+  // read before the kernel ahead of it has completed
+  pdl_wait();
+  pdl_launch_dependents();
+  prefill_body<D, G, BN>(&qmap, &kmap, &vmap, p, blockIdx.x, smem_raw);
 }
 
 template <int D>
