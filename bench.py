@@ -247,6 +247,15 @@ class GpuWorkload:
                                              out=self.out_dec if out is None else out,
                                              flags=self.pkv.DECODE_METADATA_READY)
 
+    def mixed_step(self, d=None):
+        """kv_append, then the chunk rows and the decode rows in one
+        persistent launch (pkv_paged_attn_mixed)."""
+        d = self.dev if d is None else d
+        self.pkv.pkv_kv_append(d["k_new"], d["v_new"], d["slots"], self.k_pool, self.v_pool)
+        self.pkv.pkv_paged_attn_mixed(d["q_pre"], d["cu_q"], d["ctx_pre"], d["pt_pre"], self.max_q, d["q_dec"],
+                                      d["pt_dec"], d["len_dec"], self.k_pool, self.v_pool, self.w.scale,
+                                      workspace=self.ws, out_pre=self.out_pre, out_dec=self.out_dec)
+
     def step(self, d, outs=None):
         """One pass of the hot path on device buffers d: kv_append of the
         step's new rows, then the prefill and decode calls; outs picks the
@@ -415,6 +424,9 @@ def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
         dec_ms, _ = timed(torch, g.decode_call, steps, dist)
     if g.pre:
         pre_ms, _ = timed(torch, g.prefill_call, steps, dist)
+    mixed_ms = None
+    if g.pre and g.dec and w.notes.get("attention") != "verify":
+        mixed_ms, _ = timed(torch, g.mixed_step, steps, dist)
     # end-to-end through the public API with host buffers
     g.run_e2e(warmup)
     torch.cuda.synchronize()
@@ -433,7 +445,7 @@ def measure(pkv, torch, name, steps, warmup, dist=None, clocks_index=0):
     h2d, d2h = g.io_bytes()
     res = {
         "w": w, "ms_per_step": step_ms, "e2e_ms_per_step": e2e_ms / steps,
-        "dec_ms": dec_ms, "pre_ms": pre_ms,
+        "dec_ms": dec_ms, "pre_ms": pre_ms, "mixed_ms": mixed_ms,
         "kv_bytes_dec": w.kv_bytes_read(w.decode_ids), "kv_bytes_pre": w.kv_bytes_read(w.prefill_ids),
         "tokens": int(w.new_lens.sum()), "flops_pre": prefill_flops(w),
         "launches": g.launches_per_step(), "clocks": clk.summary(), "h2d": h2d, "d2h": d2h,
@@ -684,6 +696,10 @@ def main():
             tfs = r["flops_pre"] / (r["pre_ms"] / 1e3) / 1e12
             e.update({"prefill_ms": r["pre_ms"], "prefill_flops": r["flops_pre"],
                       "prefill_tflops": tfs, "prefill_frac_of_measured_bf16": tfs / tf_sust})
+        if r["mixed_ms"]:
+            e.update({"one_launch_ms_per_step": r["mixed_ms"],
+                      "one_launch_tokens_per_s": world * r["tokens"] / (r["mixed_ms"] / 1e3),
+                      "one_launch": "kv_append + pkv_paged_attn_mixed (chunks and decode from one work queue)"})
         e["step_kv_gbs"] = (r["kv_bytes_dec"] + r["kv_bytes_pre"]) / (r["ms_per_step"] / 1e3) / 1e9
         e["clocks"] = r["clocks"]
         extra[n] = e
