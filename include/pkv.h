@@ -247,7 +247,8 @@ PKV_API int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_le
 /*
  * pkv_verify_workspace_bytes -- bytes of workspace pkv_paged_attn_verify
  * needs for total_q chunk rows whose requests hold at most max_kv_len keys
- * (pass max_pages * page_size); partition_tokens as in the call.
+ * (pass max_pages * page_size); partition_tokens as in the call (0: sized
+ * for the smallest partition the automatic choice can take, 512 keys).
  */
 PKV_API size_t pkv_verify_workspace_bytes(int32_t total_q, int32_t num_q_heads, int32_t head_dim,
                                           int32_t max_kv_len, int32_t partition_tokens);
@@ -264,9 +265,12 @@ PKV_API size_t pkv_verify_workspace_bytes(int32_t total_q, int32_t num_q_heads, 
  * partition_tokens, each handled by its own CTAs on the tensor cores, and
  * the partials are merged by pkv_split_k_combine's rule in a second kernel.
  *
- *   partition_tokens  0 = automatic (about four partitions per request of
- *               max_pages * page_size keys, within [512, 4096]), else a
- *               multiple of 64
+ *   partition_tokens  0 = automatic: no split while the (request, KV head,
+ *               128-row query tile) units number at least two per SM (each
+ *               CTA slot already has a unit; splitting would only add
+ *               partial writes), else the fewest splits of max_pages *
+ *               page_size keys that give every slot a unit, none shorter
+ *               than 512 keys; otherwise a multiple of 64
  *   workspace   device scratch of pkv_verify_workspace_bytes(...) bytes,
  *               256-byte aligned; no zeroing needed (the call clears what it
  *               needs on `stream`); calls sharing it must not overlap

@@ -318,11 +318,26 @@ int dispatch_prefill_group(int group, const pkv::prefill::Params& prm, const CUt
 // multiple of the key tile, within [512, 4096] keys.
 constexpr int kPrefillBN = pkv::prefill::kKeyTile;
 
-int32_t verify_partition(int32_t max_kv_len, int32_t partition_tokens) {
+// The smallest partition the automatic choice takes: the workspace of an
+// automatic call is sized for it.
+constexpr int32_t kVerifyMinPartition = 512;
+
+int32_t round_up_tile(long long keys) {
+  return static_cast<int32_t>((std::max<long long>(keys, 1) + kPrefillBN - 1) / kPrefillBN * kPrefillBN);
+}
+
+// Keys per split of a verify call.  Automatic: no split while the (request,
+// KV head, query tile) units already give every CTA slot of the GPU (two per
+// SM) its own unit -- splitting then only adds partial writes and CTA start-up
+// per split -- else enough splits of the longest request to fill the slots,
+// none shorter than kVerifyMinPartition keys.
+int32_t verify_partition(int32_t max_kv_len, int32_t partition_tokens, long long units, long long slots) {
   if (partition_tokens > 0) return partition_tokens;
-  const int32_t quarter = (std::max<int32_t>(max_kv_len, 1) + 3) / 4;
-  const int32_t part = (quarter + kPrefillBN - 1) / kPrefillBN * kPrefillBN;
-  return std::min<int32_t>(4096, std::max<int32_t>(512, part));
+  const int32_t whole = round_up_tile(max_kv_len);
+  if (units >= slots) return whole;
+  const long long splits = (slots + std::max<long long>(units, 1) - 1) / std::max<long long>(units, 1);
+  const int32_t part = round_up_tile((static_cast<long long>(max_kv_len) + splits - 1) / splits);
+  return std::min(whole, std::max(kVerifyMinPartition, part));
 }
 
 struct VerifyLayout {
@@ -330,9 +345,10 @@ struct VerifyLayout {
   size_t num_splits = 0, part_lse = 0, part_o = 0, total = 0;
 };
 
-VerifyLayout verify_layout(int32_t total_q, int32_t Hq, int32_t D, int32_t max_kv_len, int32_t partition_tokens) {
+// The workspace layout for splits of `partition` keys (> 0).
+VerifyLayout verify_layout(int32_t total_q, int32_t Hq, int32_t D, int32_t max_kv_len, int32_t partition) {
   VerifyLayout v;
-  v.partition = verify_partition(max_kv_len, partition_tokens);
+  v.partition = partition;
   v.splits = std::max<int32_t>(1, (max_kv_len + v.partition - 1) / v.partition);
   const size_t rows = static_cast<size_t>(total_q) * Hq;
   v.num_splits = 0;
@@ -424,13 +440,22 @@ int run_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t 
   if (st != PKV_OK) return st;
   VerifyLayout vl;
   if (split_tokens != 0) {
-    vl = verify_layout(total_q, num_q_heads, pool.head_dim, max_pages * pool.page_size,
-                       split_tokens < 0 ? 0 : split_tokens);
-    if (workspace == nullptr || workspace_bytes < vl.total) return PKV_ERR_WORKSPACE;
+    // the workspace an automatic call needs is sized for its smallest partition
+    const int32_t max_kv = max_pages * pool.page_size;
+    const VerifyLayout worst = verify_layout(total_q, num_q_heads, pool.head_dim, max_kv,
+                                             split_tokens < 0 ? std::min(kVerifyMinPartition, round_up_tile(max_kv))
+                                                              : split_tokens);
+    if (workspace == nullptr || workspace_bytes < worst.total) return PKV_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
   }
   DeviceInfo dev;
   if ((st = current_device(&dev)) != PKV_OK) return st;
+  if (split_tokens != 0) {
+    const long long units = static_cast<long long>(pl.prm.qtiles) * pool.num_kv_heads * batch;
+    vl = verify_layout(total_q, num_q_heads, pool.head_dim, max_pages * pool.page_size,
+                       verify_partition(max_pages * pool.page_size, split_tokens < 0 ? 0 : split_tokens, units,
+                                        2ll * dev.sm_count));
+  }
   if ((st = make_prefill_maps(q, k_pool, v_pool, pool, num_q_heads, total_q, &pl)) != PKV_OK) return st;
   const int D = pool.head_dim;
   pkv::prefill::Params& prm = pl.prm;
@@ -447,9 +472,10 @@ int run_prefill(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t 
   }
   st = D == 128 ? dispatch_prefill_group<128>(pl.group, prm, pl.qmap, pl.kmap, pl.vmap, max_q_len, s)
                 : dispatch_prefill_group<64>(pl.group, prm, pl.qmap, pl.kmap, pl.vmap, max_q_len, s);
-  if (st != PKV_OK || split_tokens == 0) return st;
+  if (st != PKV_OK || split_tokens == 0 || prm.splits == 1) return st;
   // merge the rows whose request was split (rows of single-split requests
-  // were written by the kernel itself)
+  // were written by the kernel itself; with one split for every request
+  // there is nothing to merge and no combine launch)
   if (D == 128)
     return launch_combine<128>(prm.part_o, prm.part_lse, prm.num_splits, total_q, num_q_heads, prm.splits,
                                prm.out, nullptr, 1, true, s);
@@ -700,7 +726,10 @@ int pkv_paged_attn_chunked_prefill(const void* q, const int32_t* cu_q_lens, int3
 size_t pkv_verify_workspace_bytes(int32_t total_q, int32_t num_q_heads, int32_t head_dim, int32_t max_kv_len,
                                   int32_t partition_tokens) {
   if (total_q < 0 || num_q_heads < 0 || head_dim < 0 || max_kv_len < 0 || partition_tokens < 0) return 0;
-  return verify_layout(total_q, num_q_heads, head_dim, max_kv_len, partition_tokens).total;
+  return verify_layout(total_q, num_q_heads, head_dim, max_kv_len,
+                       partition_tokens > 0 ? partition_tokens
+                                            : std::min(kVerifyMinPartition, round_up_tile(max_kv_len)))
+      .total;
 }
 
 int pkv_paged_attn_verify(const void* q, const int32_t* cu_q_lens, int32_t batch, int32_t num_q_heads,

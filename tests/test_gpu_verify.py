@@ -105,3 +105,40 @@ def test_verify_rows_past_the_chunks_untouched(pkv):
                               partition_tokens=512, out=out)
     assert (out[total:] == 5.0).all()
     assert pkv.pkv_device_error_flags(clear=True) == 0
+
+
+def _splits_of_rows(pkv, w, ds, total_q, max_q):
+    """Run the automatic verify call on an explicit workspace and return the
+    splits the call gave each chunk row (the workspace's leading int32s)."""
+    max_kv = ds.pt_pre.shape[1] * w.page_size
+    ws = pkv.verify_workspace(total_q, w.num_q_heads, w.head_dim, max_kv, 0, ds.q_pre.device)
+    out = torch.empty_like(ds.q_pre)
+    pkv.pkv_paged_attn_verify(ds.q_pre, ds.cu_q, ds.ctx_pre, ds.k_pool, ds.v_pool, ds.pt_pre, w.scale, max_q,
+                              partition_tokens=0, workspace=ws, out=out)
+    torch.cuda.synchronize()
+    return out, ws[: total_q * 4].view(torch.int32).cpu().numpy()
+
+
+def test_verify_automatic_split_choice(pkv):
+    # few (request, KV head) units: the automatic partition splits the long
+    # requests so that the GPU's CTA slots fill; many units: no split at all
+    slots = 2 * torch.cuda.get_device_properties(0).multi_processor_count
+    few = make_workload("mixed_prefill_decode", 9, n_prefill=3, chunks=[4, 4, 2], ctxs=[20000, 9000, 100],
+                        n_decode=1)
+    assert few.num_kv_heads * 3 < slots
+    many = make_workload("spec_verify", 1)
+    assert many.num_kv_heads * len(many.prefill_ids) >= slots
+    for w, expect_split in ((few, True), (many, False)):
+        ds, os_ = DeviceStep(pkv, w), OracleStep(w)
+        ds.append()
+        os_.append()
+        ref, _, rows = os_.prefill()
+        pre = list(w.prefill_ids)
+        total_q, max_q = int(w.new_lens[pre].sum()), int(w.new_lens[pre].max())
+        out, splits = _splits_of_rows(pkv, w, ds, total_q, max_q)
+        assert_close(bf16_to_f64(out)[rows], ref[rows], f"automatic verify ({'few' if expect_split else 'many'})")
+        if expect_split:
+            assert splits.max() > 1 and splits.min() >= 1
+        else:
+            assert (splits == 1).all()
+        assert pkv.pkv_device_error_flags(clear=True) == 0
