@@ -312,10 +312,9 @@ int dispatch_prefill_group(int group, const pkv::prefill::Params& prm, const CUt
   return PKV_ERR_UNSUPPORTED;
 }
 
-// Split-K chunk attention (short chunks over long contexts): the automatic
-// partition depends on the longest context only, so the workspace size can
-// be computed without device data: about four splits per request, a
-// multiple of the key tile, within [512, 4096] keys.
+// Split-K chunk attention (short chunks over long contexts).  The workspace
+// size depends on the longest context and the partition only, so it can be
+// computed without device data.
 constexpr int kPrefillBN = pkv::prefill::kKeyTile;
 
 // The smallest partition the automatic choice takes: the workspace of an
