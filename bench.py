@@ -8,7 +8,8 @@ fragmented large batch, tiny decode).
 
 A step is one pass of the hot path over one batch: kv_append of the step's new
 K/V rows, then attention (chunked prefill for prompt chunks, decode with its
-split-K partition and in-kernel merge for decode rows).  Inputs are resident in HBM
+split-K partition and in-kernel merge for decode rows); a decode-only batch
+appends and decodes in one launch (pkv_paged_attn_decode_append).  Inputs are resident in HBM
 when the timed region starts; the KV a step reads is larger than the 126 MB
 L2, so no flush is needed between steps.  Under torchrun each rank runs its
 own batch (requests shard across GPUs with no data-path collective: weak
@@ -193,6 +194,13 @@ class GpuWorkload:
         self.dev = self.in_dev[0].views
         self.dev_sets = [d.views for d in self.in_dev]
         self.dec, self.pre = dec, pre
+        # a decode-only step whose new rows are one per request, each at its
+        # request's position kv_lens - 1, is appended and decoded in one
+        # launch (pkv_paged_attn_decode_append)
+        last = np.array([int(w.page_table[r][(int(w.kv_lens[r]) - 1) // w.page_size]) * w.page_size
+                         + (int(w.kv_lens[r]) - 1) % w.page_size for r in dec], np.int64)
+        self.fused = (not pre and len(dec) == w.B and len(s) == len(dec) and bool((w.kv_lens[dec] > 0).all())
+                      and np.array_equal(np.asarray(s, np.int64), last))
         self.max_q = int(w.new_lens[pre].max()) if pre else 0
         if dec:
             self.ws = pkv.decode_workspace(len(dec), w.num_q_heads, w.head_dim,
@@ -223,7 +231,10 @@ class GpuWorkload:
 
     def launches_per_step(self):
         # kv_append, the decode partition kernel (the automatic split merges
-        # in-kernel, no combine launch), the prefill kernel
+        # in-kernel, no combine launch), the prefill kernel; a fused decode
+        # step is the partition kernel alone
+        if self.fused:
+            return 1
         return 1 + (1 if self.dec else 0) + (1 if self.pre else 0)
 
     def prefill_call(self, d=None, out=None):
@@ -258,8 +269,17 @@ class GpuWorkload:
 
     def step(self, d, outs=None):
         """One pass of the hot path on device buffers d: kv_append of the
-        step's new rows, then the prefill and decode calls; outs picks the
-        output buffers (default: the first set)."""
+        step's new rows, then the prefill and decode calls (for a decode-only
+        step, both in one fused launch); outs picks the output buffers
+        (default: the first set)."""
+        if self.fused:
+            # the kernel just ahead (the previous step's) writes neither
+            # lengths nor page tables
+            self.pkv.pkv_paged_attn_decode_append(
+                d["q_dec"], d["k_new"], d["v_new"], self.k_pool, self.v_pool, d["pt_dec"], d["len_dec"],
+                self.w.scale, 0, workspace=self.ws, out=outs["dec"] if outs is not None else self.out_dec,
+                flags=self.pkv.DECODE_METADATA_READY)
+            return
         self.pkv.pkv_kv_append(d["k_new"], d["v_new"], d["slots"], self.k_pool, self.v_pool)
         if self.pre:
             self.prefill_call(d, outs["pre"] if outs is not None else None)

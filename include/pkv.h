@@ -197,6 +197,37 @@ PKV_API int pkv_paged_attn_decode_flags(const void* q, int32_t batch, int32_t nu
                                         float* out_lse, uint32_t flags, pkv_stream_t stream);
 
 /*
+ * pkv_paged_attn_decode_append -- one decode step's kv_append and decode in
+ * one launch (the decode step of the tiny-llm source reading, "Paged KV
+ * Cache": the new token's K/V row goes into its page, then the query
+ * attends to the whole context including it).  Request r's new row
+ * (k_new[r], v_new[r]) is the key and value of position kv_lens[r] - 1: the
+ * warp that streams that position reads it from k_new / v_new instead of the
+ * pool and writes it bit for bit to its pool slot (page_table[r][(kv_lens[r]
+ * - 1) / page_size], row (kv_lens[r] - 1) % page_size).  The result equals
+ * pkv_kv_append of those rows at those slots followed by
+ * pkv_paged_attn_decode_flags, up to the summation order of the last key.
+ *
+ *   k_new, v_new   [batch][Hkv][d] bf16, 16-byte aligned; read only
+ *   k_pool, v_pool written at the batch's new slots only
+ *   other arguments as pkv_paged_attn_decode_flags
+ *
+ * Requests with kv_lens[r] = 0 append nothing.  A new row whose page id is
+ * out of range, or whose kv_lens is out of range, is not written (the call
+ * raises PKV_FLAG_BAD_PAGE or PKV_FLAG_BAD_LENGTH as decode does).  No two
+ * requests may share the slot of their new rows.  PKV_ERR_UNSUPPORTED in a
+ * build that streams pages with bulk copies (PKV_DECODE_CPASYNC=0).
+ */
+PKV_API int pkv_paged_attn_decode_append(const void* q, const void* k_new, const void* v_new,
+                                         int32_t batch, int32_t num_q_heads, void* k_pool,
+                                         void* v_pool, pkv_pool_desc pool,
+                                         const int32_t* page_table, int32_t max_pages,
+                                         const int32_t* kv_lens, float scale,
+                                         int32_t partition_tokens, void* workspace,
+                                         size_t workspace_bytes, void* out, float* out_lse,
+                                         uint32_t flags, pkv_stream_t stream);
+
+/*
  * pkv_split_k_combine -- merge split-K partials by their log-sum-exp weights
  * (mini-vllm advanced series design, adv04 "Flash-Decoding"; the formula is
  * the plain reading: M = max_s lse_s, w_s = exp(lse_s - M),

@@ -30,6 +30,7 @@ __all__ = [
     "pkv_paged_attn_decode_static", "pkv_qk_norm_rope_append", "pkv_kv_append_cow",
     "pkv_verify_workspace_bytes", "verify_workspace", "pkv_paged_attn_verify", "pkv_paged_attn_decode_flags",
     "DECODE_METADATA_READY", "pkv_mixed_workspace_bytes", "mixed_workspace", "pkv_paged_attn_mixed",
+    "pkv_paged_attn_decode_append",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -85,6 +86,9 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_attn_decode_flags.argtypes = [P, I32, I32, P, P, _PoolDesc, P, I32, P, F32, I32, P, SZ,
                                                 P, P, ctypes.c_uint32, P]
     lib.pkv_paged_attn_decode_flags.restype = ctypes.c_int
+    lib.pkv_paged_attn_decode_append.argtypes = [P, P, P, I32, I32, P, P, _PoolDesc, P, I32, P, F32, I32, P, SZ,
+                                                 P, P, ctypes.c_uint32, P]
+    lib.pkv_paged_attn_decode_append.restype = ctypes.c_int
     lib.pkv_mixed_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.pkv_mixed_workspace_bytes.restype = SZ
     lib.pkv_paged_attn_mixed.argtypes = [P, P, I32, I32, I32, P, P, I32, P, I32, P, I32, P, I32, P, P, _PoolDesc,
@@ -211,6 +215,39 @@ def pkv_paged_attn_decode_flags(q, k_pool, v_pool, page_table, kv_lens, scale, p
     _check("pkv_paged_attn_decode_flags", _lib.pkv_paged_attn_decode_flags(
         _ptr(q), B, hq, _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(page_table),
         max_pages, _ptr(kv_lens), float(scale), int(partition_tokens), _ptr(workspace),
+        workspace.numel(), _ptr(out), _ptr(out_lse), int(flags), _stream(stream)))
+    return out
+
+
+def pkv_paged_attn_decode_append(q, k_new, v_new, k_pool, v_pool, page_table, kv_lens, scale, partition_tokens=0,
+                                 workspace=None, out=None, out_lse=None, flags=0, stream=None):
+    """One decode step in one launch: request r's new row (k_new[r], v_new[r],
+    [B, Hkv, d]) is written to its pool slot at position kv_lens[r] - 1 and
+    attended to as that key; otherwise as pkv_paged_attn_decode_flags."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(k_pool, "k_pool", torch.bfloat16, 4)
+    _need(v_pool, "v_pool", torch.bfloat16, 4)
+    _need(page_table, "page_table", torch.int32, 2)
+    _need(kv_lens, "kv_lens", torch.int32, 1)
+    B, hq, d = q.shape
+    max_pages = page_table.shape[1]
+    if page_table.shape[0] != B or kv_lens.shape[0] != B:
+        raise ValueError("page_table / kv_lens rows must equal the batch")
+    if tuple(k_new.shape) != (B, k_pool.shape[1], d) or k_new.shape != v_new.shape:
+        raise ValueError("k_new / v_new must be [batch, Hkv, d]")
+    if workspace is None:
+        workspace = decode_workspace(B, hq, d, max_pages * k_pool.shape[2], partition_tokens, q.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 3)
+    if out_lse is not None:
+        _need(out_lse, "out_lse", torch.float32, 2)
+    _check("pkv_paged_attn_decode_append", _lib.pkv_paged_attn_decode_append(
+        _ptr(q), _ptr(k_new), _ptr(v_new), B, hq, _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool),
+        _ptr(page_table), max_pages, _ptr(kv_lens), float(scale), int(partition_tokens), _ptr(workspace),
         workspace.numel(), _ptr(out), _ptr(out_lse), int(flags), _stream(stream)))
     return out
 

@@ -552,20 +552,26 @@ pkv::decode::Params fill_decode(const void* q, int32_t batch, int32_t num_q_head
   prm.merge_nodes = dp.ss.nodes;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.meta_ready = (flags & PKV_DECODE_METADATA_READY) ? 1 : 0;
+  prm.k_new = nullptr;
+  prm.v_new = nullptr;
   return prm;
 }
 
 // Launch a checked decode call on workspace ws (at least dp.wl.total bytes,
-// 256-byte aligned).
+// 256-byte aligned); k_new / v_new: the step's new rows to append and attend
+// to (one per request), or null.
 int run_decode(const void* q, int32_t batch, int32_t num_q_heads, const void* k_pool, const void* v_pool,
                const pkv_pool_desc& pool, const int32_t* page_table, int32_t max_pages,
                const int32_t* kv_lens, float scale, int32_t partition_tokens, const DecodePlan& dp,
-               void* workspace, void* out, float* out_lse, uint32_t flags, cudaStream_t s) {
+               void* workspace, void* out, float* out_lse, uint32_t flags, cudaStream_t s,
+               const void* k_new = nullptr, const void* v_new = nullptr) {
   DeviceInfo dev;
   int st;
   if ((st = current_device(&dev)) != PKV_OK) return st;
-  const pkv::decode::Params prm = fill_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages,
-                                              kv_lens, scale, partition_tokens, dp, workspace, out, out_lse, flags);
+  pkv::decode::Params prm = fill_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens,
+                                        scale, partition_tokens, dp, workspace, out, out_lse, flags);
+  prm.k_new = static_cast<const uint16_t*>(k_new);
+  prm.v_new = static_cast<const uint16_t*>(v_new);
   if ((st = prepare_workspace(workspace, dp.wl.zero_bytes, s)) != PKV_OK) return st;
   if (pool.head_dim == 128) return dispatch_decode_group<128>(dp.group, prm, dev.sm_count, s);
   return dispatch_decode_group<64>(dp.group, prm, dev.sm_count, s);
@@ -692,6 +698,26 @@ int pkv_paged_attn_decode_flags(const void* q, int32_t batch, int32_t num_q_head
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
   return run_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens, scale,
                     partition_tokens, dp, workspace, out, out_lse, flags, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int pkv_paged_attn_decode_append(const void* q, const void* k_new, const void* v_new, int32_t batch,
+                                 int32_t num_q_heads, void* k_pool, void* v_pool, pkv_pool_desc pool,
+                                 const int32_t* page_table, int32_t max_pages, const int32_t* kv_lens, float scale,
+                                 int32_t partition_tokens, void* workspace, size_t workspace_bytes, void* out,
+                                 float* out_lse, uint32_t flags, pkv_stream_t stream) {
+  if ((flags & ~static_cast<uint32_t>(PKV_DECODE_METADATA_READY)) != 0) return PKV_ERR_BAD_SHAPE;
+  DecodePlan dp;
+  const int st = check_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens,
+                              scale, partition_tokens, out, &dp);
+  if (st != PKV_OK || batch == 0) return st;
+  if (!k_new || !v_new) return PKV_ERR_NULL_POINTER;
+  if (!aligned16(k_new) || !aligned16(v_new)) return PKV_ERR_MISALIGNED;
+  if (!pkv::decode::kCpAsync) return PKV_ERR_UNSUPPORTED;  // the bulk-copy build streams rows it cannot swap
+  if (workspace == nullptr || workspace_bytes < dp.wl.total) return PKV_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  return run_decode(q, batch, num_q_heads, k_pool, v_pool, pool, page_table, max_pages, kv_lens, scale,
+                    partition_tokens, dp, workspace, out, out_lse, flags, reinterpret_cast<cudaStream_t>(stream),
+                    k_new, v_new);
 }
 
 int pkv_split_k_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,

@@ -152,6 +152,22 @@ def test_host_validation_without_gpu(lib):
     assert decf(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, ws, 1 << 20, dummy, None, 2, None) == -2
     assert decf(dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, ws, 64, dummy, None, 1, None) == -5
 
+    lib.pkv_paged_attn_decode_append.argtypes = [P, P, P, I32, I32, P, P, PoolDesc, P, I32, P, ctypes.c_float,
+                                                 I32, P, ctypes.c_size_t, P, P, ctypes.c_uint32, P]
+    deca = lib.pkv_paged_attn_decode_append
+    # unknown option bit; new rows missing; new rows misaligned; workspace too small
+    assert deca(dummy, dummy, dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, ws, 1 << 20, dummy, None,
+                2, None) == -2
+    assert deca(dummy, None, dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, ws, 1 << 20, dummy, None,
+                0, None) == -1
+    assert deca(dummy, dummy, ctypes.c_void_p(24), 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, ws,
+                1 << 20, dummy, None, 0, None) == -4
+    assert deca(dummy, dummy, dummy, 4, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, ws, 64, dummy, None, 1,
+                None) == -5
+    # an empty batch is a valid call that launches nothing
+    assert deca(None, None, None, 0, 32, dummy, dummy, good, dummy, 8, dummy, 0.1, 0, None, 0, None, None, 0,
+                None) == 0
+
     lib.pkv_paged_attn_verify.argtypes = [P, P, I32, I32, I32, I32, P, P, P, PoolDesc, P, I32, ctypes.c_float,
                                           I32, P, ctypes.c_size_t, P, P]
     ver = lib.pkv_paged_attn_verify
