@@ -392,7 +392,10 @@ __device__ __forceinline__ void merge_regs(const Params& p, int r, int g, int ns
 // `smem` is the CTA's dynamic shared memory.  kLean: 8 elements of d per
 // lane in the score phase even where 16 would fit, which frees the
 // registers of half the query rows (for kernels that hold other work).
-template <int D, int G, int NS, bool kLean = false>
+// kAppend: the launch takes each request's new row from p.k_new / p.v_new
+// and writes it to the pool (a separate instantiation, so plain decode keeps
+// its code unchanged).
+template <int D, int G, int NS, bool kLean = false, bool kAppend = false>
 __device__ __forceinline__ void decode_body(const Params& p, int cta, int ncta, int W, uint8_t* smem) {
   using LY = Layout<D, G, NS>;
   constexpr int kFI = kMergeFanIn<D>;  // merge-tree fan-in
@@ -674,7 +677,7 @@ __device__ __forceinline__ void decode_body(const Params& p, int cta, int ncta, 
         // the step's new rows given, that row comes from them, and the lanes
         // that carry it also write it to its pool slot (no other warp of the
         // launch reads that slot)
-        if (p.k_new != nullptr && (flags & kLast) && it_t0 + it_ntok == lens[it_r]) {
+        if (kAppend && (flags & kLast) && it_t0 + it_ntok == lens[it_r]) {
           const int last = ntok - 1, bl = last / CK::kBoxRows, first_piece = (last % CK::kBoxRows) * (D / 8);
           const size_t nrow = (static_cast<size_t>(it_r) * p.Hkv + it_g) * D;
           const uint8_t* knew = reinterpret_cast<const uint8_t*>(p.k_new + nrow);
@@ -1038,10 +1041,10 @@ __device__ __forceinline__ void decode_body(const Params& p, int cta, int ncta, 
   }
 }
 
-template <int D, int G, int NS, int MAXW>
+template <int D, int G, int NS, int MAXW, bool APPEND = false>
 __global__ void __launch_bounds__(MAXW * 32, 1) partition_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  decode_body<D, G, NS>(p, blockIdx.x, gridDim.x, blockDim.x >> 5, smem);
+  decode_body<D, G, NS, false, APPEND>(p, blockIdx.x, gridDim.x, blockDim.x >> 5, smem);
 }
 
 // Merge split partials.  One CTA per (request, query head) row; its warps

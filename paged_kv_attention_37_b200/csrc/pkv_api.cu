@@ -252,7 +252,9 @@ int launch_decode(const pkv::decode::Params& prm, int sm_count, cudaStream_t str
   constexpr int kMaxWD = D == 128 ? PKV_DECODE_MAXW128 : PKV_DECODE_MAXW64;
   constexpr int kMaxW = G == 8 ? (kMaxWD < 8 ? kMaxWD : 8) : kMaxWD;
   using LY = pkv::decode::Layout<D, G, NS>;
-  auto kernel = pkv::decode::partition_kernel<D, G, NS, kMaxW>;
+  // with the step's new rows: the instantiation that appends them
+  auto kernel = prm.k_new != nullptr ? pkv::decode::partition_kernel<D, G, NS, kMaxW, true>
+                                     : pkv::decode::partition_kernel<D, G, NS, kMaxW, false>;
   constexpr size_t kBudget = 227 * 1024;
   const size_t fixed = LY::bytes(0, prm.B);
   if (fixed + LY::kWarpBytes > kBudget) return PKV_ERR_BAD_SHAPE;  // batch too large for the plan
