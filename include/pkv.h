@@ -202,11 +202,12 @@ PKV_API int pkv_paged_attn_decode_flags(const void* q, int32_t batch, int32_t nu
  * Cache": the new token's K/V row goes into its page, then the query
  * attends to the whole context including it).  Request r's new row
  * (k_new[r], v_new[r]) is the key and value of position kv_lens[r] - 1: the
- * warp that streams that position reads it from k_new / v_new instead of the
- * pool and writes it bit for bit to its pool slot (page_table[r][(kv_lens[r]
- * - 1) / page_size], row (kv_lens[r] - 1) % page_size).  The result equals
+ * warp that streams that position first writes it bit for bit to its pool
+ * slot (page_table[r][(kv_lens[r] - 1) / page_size], row (kv_lens[r] - 1) %
+ * page_size), makes the write visible and then streams the page as usual;
+ * no other warp of the launch reads that slot.  The result equals
  * pkv_kv_append of those rows at those slots followed by
- * pkv_paged_attn_decode_flags, up to the summation order of the last key.
+ * pkv_paged_attn_decode_flags.
  *
  *   k_new, v_new   [batch][Hkv][d] bf16, 16-byte aligned; read only
  *   k_pool, v_pool written at the batch's new slots only

@@ -145,8 +145,8 @@ struct Params {
   float scale_log2;           // softmax scale * log2(e)
   int32_t meta_ready;         // the kernel ahead writes neither kv_lens nor page_table
   // the step's new rows, one per request ([B][Hkv][D] bf16), or null: row r
-  // is the key/value of position kv_lens[r] - 1, read from here and written
-  // to its pool slot by the warp that streams that position
+  // is the key/value of position kv_lens[r] - 1, written to its pool slot by
+  // the warp that streams that position just before it streams it
   const uint16_t* k_new;
   const uint16_t* v_new;
 };
@@ -674,50 +674,39 @@ __device__ __forceinline__ void decode_body(const Params& p, int cta, int ncta, 
       if (ntok > 0) {
         constexpr int kPieces = CK::kBoxRows * D / 8;  // 16-byte pieces per 16-row piece
         // the chunk that ends the request holds position kv_lens[r] - 1: with
-        // the step's new rows given, that row comes from them, and the lanes
-        // that carry it also write it to its pool slot (no other warp of the
-        // launch reads that slot)
-        if (kAppend && (flags & kLast) && it_t0 + it_ntok == lens[it_r]) {
-          const int last = ntok - 1, bl = last / CK::kBoxRows, first_piece = (last % CK::kBoxRows) * (D / 8);
-          const size_t nrow = (static_cast<size_t>(it_r) * p.Hkv + it_g) * D;
-          const uint8_t* knew = reinterpret_cast<const uint8_t*>(p.k_new + nrow);
-          const uint8_t* vnew = reinterpret_cast<const uint8_t*>(p.v_new + nrow);
-          // no write through a bad page id, nor for a length that was out of
-          // range (flagged above and clamped: its last row is not kv_lens - 1)
-          const bool write_pool = ((bad_boxes >> bl) & 1u) == 0 && __ldg(p.kv_lens + it_r) == lens[it_r];
+        // the step's new rows given, the warp first writes that row to its
+        // pool slot (one 16-byte piece per lane, K then V), makes the stores
+        // visible device-wide and then streams the chunk as usual; no other
+        // warp of the launch reads that slot.  A bad page id or an
+        // out-of-range length (both flagged) writes nothing.
+        if constexpr (kAppend) {
+          if ((flags & kLast) && it_t0 + it_ntok == lens[it_r]) {
+            const int last = ntok - 1, bl = last / CK::kBoxRows;
+            if (((bad_boxes >> bl) & 1u) == 0 && __ldg(p.kv_lens + it_r) == lens[it_r] && lane < D / 4) {
+              const bool is_v = lane >= D / 8;
+              const int piece = is_v ? lane - D / 8 : lane;
+              const size_t nrow = (static_cast<size_t>(it_r) * p.Hkv + it_g) * D + piece * 8;
+              size_t row_bl = 0;  // rows[bl], selected without indexing the array at run time
 #pragma unroll
-          for (int b = 0; b < CK::kBoxes; ++b) {
-            if (b >= nbox) break;
-            const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + rows[b] * D);
-            const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + rows[b] * D);
-#pragma unroll
-            for (int i = lane; i < kPieces; i += 32) {
-              const uint8_t* ks = ksrc + i * 16;
-              const uint8_t* vs = vsrc + i * 16;
-              if (b == bl && i >= first_piece && i < first_piece + D / 8) {
-                const int off = (i - first_piece) * 16;
-                if (write_pool) {
-                  *reinterpret_cast<uint4*>(const_cast<uint8_t*>(ks)) = *reinterpret_cast<const uint4*>(knew + off);
-                  *reinterpret_cast<uint4*>(const_cast<uint8_t*>(vs)) = *reinterpret_cast<const uint4*>(vnew + off);
-                }
-                ks = knew + off;
-                vs = vnew + off;
-              }
-              cp_async16(st + b * (CK::kBoxRows * D * 2) + i * 16, ks);
-              cp_async16(st + LY::kKBytes + b * (CK::kBoxRows * D * 2) + i * 16, vs);
+              for (int b = 0; b < CK::kBoxes; ++b)
+                if (b == bl) row_bl = rows[b];
+              const size_t prow = (row_bl + last % CK::kBoxRows) * D + piece * 8;
+              const uint4 val = *reinterpret_cast<const uint4*>((is_v ? p.v_new : p.k_new) + nrow);
+              *reinterpret_cast<uint4*>(const_cast<uint16_t*>(is_v ? p.v_pool : p.k_pool) + prow) = val;
+              __threadfence();
             }
+            __syncwarp();
           }
-        } else {
+        }
 #pragma unroll
-          for (int b = 0; b < CK::kBoxes; ++b) {
-            if (b >= nbox) break;
-            const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + rows[b] * D);
-            const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + rows[b] * D);
+        for (int b = 0; b < CK::kBoxes; ++b) {
+          if (b >= nbox) break;
+          const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + rows[b] * D);
+          const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + rows[b] * D);
 #pragma unroll
-            for (int i = lane; i < kPieces; i += 32) {
-              cp_async16(st + b * (CK::kBoxRows * D * 2) + i * 16, ksrc + i * 16);
-              cp_async16(st + LY::kKBytes + b * (CK::kBoxRows * D * 2) + i * 16, vsrc + i * 16);
-            }
+          for (int i = lane; i < kPieces; i += 32) {
+            cp_async16(st + b * (CK::kBoxRows * D * 2) + i * 16, ksrc + i * 16);
+            cp_async16(st + LY::kKBytes + b * (CK::kBoxRows * D * 2) + i * 16, vsrc + i * 16);
           }
         }
         if (it_k == 0) {
