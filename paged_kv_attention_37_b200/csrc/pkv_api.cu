@@ -297,7 +297,7 @@ int launch_prefill(const pkv::prefill::Params& prm, const CUtensorMap& qmap, con
   if (blocks > 0x7FFFFFFFll) return PKV_ERR_BAD_SHAPE;
   pkv::prefill::Params args = prm;
   args.qtiles = static_cast<int32_t>(tiles);
-  return launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(pkv::prefill::kThreads), smem, stream, qmap,
+  return launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(pkv::prefill::kThreadsAlone), smem, stream, qmap,
                     kmap, vmap, args);
 }
 

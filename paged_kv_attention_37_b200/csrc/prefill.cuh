@@ -30,7 +30,8 @@ namespace pkv {
 namespace prefill {
 
 constexpr int kM = 128;  // query rows per CTA
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;        // TMA warp, MMA warp, 4 softmax warps (chunk units of the mixed kernel)
+constexpr int kThreadsAlone = 224;   // the standalone kernel: S and P.V issued by two warps
 // What the launcher needs to know: query rows (positions x group heads) per
 // CTA, keys per K/V tile (split partitions are multiples of it), and the
 // dynamic shared memory of a CTA.
@@ -120,7 +121,11 @@ __device__ __forceinline__ int request_by_weight(const Params& p, int rank) {
 // memory `smem_raw`.  The caller has waited for the kernel ahead.  kOnce: the
 // CTA runs one unit and gives up its TMEM allocation permit after it
 // allocates; a persistent CTA (one allocation per unit) keeps it.
-template <int D, int G, int BN, bool kOnce = true>
+// kTwoIssuers: warp 1 issues the S MMAs and warp 2 the P.V MMAs (softmax
+// warps 3..6); else warp 1 issues both (softmax warps 2..5).  One thread
+// issues tcgen05.mma at a bounded rate, so two issuers per CTA keep the
+// tensor pipe busier.
+template <int D, int G, int BN, bool kOnce = true, bool kTwoIssuers = false>
 __device__ __forceinline__ void prefill_body(const CUtensorMap* qmap_p, const CUtensorMap* kmap_p,
                                              const CUtensorMap* vmap_p, const Params& p, int unit,
                                              uint8_t* smem_raw) {
@@ -194,7 +199,7 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap* qmap_p, const CU
       mbar_init(bar(kPFull + i), 128);
       mbar_init(bar(kPVDone + i), 1);
     }
-    mbar_init(bar(kFinal), 1);
+    mbar_init(bar(kFinal), kTwoIssuers ? 2 : 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -283,6 +288,50 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap* qmap_p, const CU
       pg_prev = pg;
       __syncwarp();
     }
+  } else if (kTwoIssuers && (warp == 1 || warp == 2)) {
+    // ======================== MMA issuers (S / P.V) ========================
+    // warp 1: S of tile j once K(j) is in and the buffer's P.V(j-2) is done;
+    // warp 2: P.V of tile i once P(i) and V(i) are in
+    bool ok = mbar_wait(bar(kQ), 0);
+    if (warp == 1) {
+      for (int j = 0; j < nt && ok; ++j) {
+        const int b = j & 1;
+        ok = (j < 2 || mbar_wait(bar(kPVDone + b), ((j - 2) >> 1) & 1)) && mbar_wait(bar(kKFull + b), (j >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after_sync();
+        if (lane == 0) {
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t a = smem_desc_sw128(sQ + (ks >> 2) * LY::kQHalf + (ks & 3) * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(sK(b) + (ks >> 2) * LY::kKVHalf + (ks & 3) * 32, 16, 1024);
+            tc_mma_ss(tmem + (b ? kColS1 : kColS0), a, bdesc, kIdescS, ks > 0);
+          }
+          tc_commit(bar(kSFull + b));
+          tc_commit(bar(kKEmpty + b));
+        }
+        __syncwarp();
+      }
+    } else {
+      for (int i = 0; i < nt && ok; ++i) {
+        const int b = i & 1;
+        ok = mbar_wait(bar(kPFull + b), (i >> 1) & 1) && mbar_wait(bar(kVFull + b), (i >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after_sync();
+        if (lane == 0) {
+#pragma unroll
+          for (int ks = 0; ks < kN / 16; ++ks) {
+            const uint32_t a = tmem + (b ? kColS1 : kColS0) + ks * 8;
+            const uint64_t bdesc = smem_desc_sw128(sV(b) + ks * 16 * 128, LY::kKVHalf, 1024);
+            tc_mma_ts(tmem + kColO, a, bdesc, kIdescPV, i > 0 || ks > 0);
+          }
+          tc_commit(bar(kPVDone + b));
+          tc_commit(bar(kVEmpty + b));
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0) tc_commit(bar(kFinal));
+    __syncwarp();
   } else if (warp == 1) {
     // ============================ MMA issuer =============================
     // Two streams of MMAs: S of tile j (needs K(j) and a free S buffer) and
@@ -355,6 +404,7 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap* qmap_p, const CU
   } else {
     // ========================= softmax / epilogue ========================
     const int quad = warp & 3;             // TMEM lane quadrant this warp may access
+    const int sw = warp - (kTwoIssuers ? 3 : 2);  // 0..3 within the softmax warps (ragged-tile zeroing)
     const int row = quad * 32 + lane;      // query row of this thread
     const int pos_local = row / G, hh = row % G;
     const int qpos = pos_lo + pos_local;   // absolute position
@@ -453,7 +503,7 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap* qmap_p, const CU
         const int nbytes = (kN - first) * 128;
         for (int h = 0; h < D / 64; ++h) {
           uint8_t* vz = smem + LY::kVOff + b * LY::kKVTile + h * LY::kKVHalf + first * 128;
-          for (int off = (row) * 16; off < nbytes; off += kM * 16)
+          for (int off = (sw * 32 + lane) * 16; off < nbytes; off += kM * 16)
             *reinterpret_cast<uint4*>(vz + off) = make_uint4(0, 0, 0, 0);
         }
       }
@@ -523,7 +573,7 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap* qmap_p, const CU
 }
 
 template <int D, int G, int BN>
-__global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
+__global__ void __launch_bounds__(kThreadsAlone, BN == 64 ? 2 : 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -531,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
   // read before the kernel ahead of it has completed
   pdl_wait();
   pdl_launch_dependents();
-  prefill_body<D, G, BN>(&qmap, &kmap, &vmap, p, blockIdx.x, smem_raw);
+  prefill_body<D, G, BN, true, true>(&qmap, &kmap, &vmap, p, blockIdx.x, smem_raw);
 }
 
 template <int D>
