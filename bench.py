@@ -138,6 +138,19 @@ class Packed:
             self.views[k] = self.buf[offs[k]:offs[k] + nb].view(dt).view(shape)
 
 
+def fusable_decode_step(w, slots) -> bool:
+    """True when a step of workload w is decode only and its new rows (with
+    slot mapping `slots`, in request order) are one per request, each at its
+    request's position kv_lens - 1: the rows pkv_paged_attn_decode_append
+    appends itself."""
+    dec, pre = list(w.decode_ids), list(w.prefill_ids)
+    if pre or len(dec) != w.B or len(slots) != len(dec) or not bool((w.kv_lens[dec] > 0).all()):
+        return False
+    last = np.array([int(w.page_table[r][(int(w.kv_lens[r]) - 1) // w.page_size]) * w.page_size
+                     + (int(w.kv_lens[r]) - 1) % w.page_size for r in dec], np.int64)
+    return bool(np.array_equal(np.asarray(slots, np.int64), last))
+
+
 class GpuWorkload:
     """Device buffers for one workload: pools with every request's context
     (drawn on the GPU, seeded), and the step's inputs (host-generated)."""
@@ -197,10 +210,7 @@ class GpuWorkload:
         # a decode-only step whose new rows are one per request, each at its
         # request's position kv_lens - 1, is appended and decoded in one
         # launch (pkv_paged_attn_decode_append)
-        last = np.array([int(w.page_table[r][(int(w.kv_lens[r]) - 1) // w.page_size]) * w.page_size
-                         + (int(w.kv_lens[r]) - 1) % w.page_size for r in dec], np.int64)
-        self.fused = (not pre and len(dec) == w.B and len(s) == len(dec) and bool((w.kv_lens[dec] > 0).all())
-                      and np.array_equal(np.asarray(s, np.int64), last))
+        self.fused = fusable_decode_step(w, s)
         self.max_q = int(w.new_lens[pre].max()) if pre else 0
         if dec:
             self.ws = pkv.decode_workspace(len(dec), w.num_q_heads, w.head_dim,

@@ -179,6 +179,10 @@ def test_host_validation_without_gpu(lib):
     # rows x heads x splits partials of d fp32 and their lse, about four splits
     assert lib.pkv_verify_workspace_bytes(256, 32, 128, 4096, 0) >= 256 * 32 * 4 * 129 * 4
     assert lib.pkv_verify_workspace_bytes(-1, 32, 128, 4096, 0) == 0
+    # the automatic choice never cuts finer than 512 keys, and its workspace
+    # is sized for exactly that (a context under 512 keys: one split)
+    assert lib.pkv_verify_workspace_bytes(256, 32, 128, 4096, 0) == lib.pkv_verify_workspace_bytes(256, 32, 128, 4096, 512)
+    assert lib.pkv_verify_workspace_bytes(16, 8, 64, 300, 0) == lib.pkv_verify_workspace_bytes(16, 8, 64, 300, 320)
 
     lib.pkv_qk_norm_rope_append.argtypes = [P, P, P, I32, I32, P, P, P, P, ctypes.c_float, ctypes.c_float,
                                             P, P, P, PoolDesc, P]
