@@ -295,7 +295,8 @@ PKV_API size_t pkv_verify_workspace_bytes(int32_t total_q, int32_t num_q_heads, 
  * of request r sits at ctx_offsets[r] + i and sees keys 0 .. ctx_offsets[r]
  * + i); the keys of each request are cut into partitions of
  * partition_tokens, each handled by its own CTAs on the tensor cores, and
- * the partials are merged by pkv_split_k_combine's rule in a second kernel.
+ * the partials of split requests are merged by pkv_split_k_combine's rule in
+ * a second kernel (not launched when no request is split).
  *
  *   partition_tokens  0 = automatic: no split while the (request, KV head,
  *               128-row query tile) units number at least two per SM (each
